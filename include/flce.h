@@ -1,0 +1,163 @@
+/*
+ * flce.h - C ABI of the B200 (sm_100a) fused LM-head projection + cross-entropy.
+ *
+ * The operation (NeMo-AutoModel pages "nemo_automodel.components.loss.linear_ce",
+ * FusedLinearCrossEntropy, and "nemo_automodel.components.models.inkling2.loss",
+ * Inkling2FusedLinearCrossEntropy, class docstring):
+ *
+ *   z[n, v]  = sum_h hidden[n, h] * Wb[v, h]            BF16 x BF16, FP32 accumulate
+ *   zc[n, v] = c * tanh(z[n, v] / c)  (c > 0), else z   FP32 logit softcap
+ *   lse[n]   = log sum_{v < V} exp(zc[n, v])            rows >= V never enter the softmax
+ *   l[n]     = lse[n] - zc[n, y_n]  if y_n != ignore_index, else 0
+ *   loss     = sum_n l[n]  (/ num_label_tokens if > 0),  or mean, or per token
+ *
+ * with Wb = the first V = unpadded_vocab rows of the head, rounded to BF16 (RNE)
+ * when the head is FP32 (inkling2 page: "An FP32 head is rounded to BF16").
+ * The backward recomputes the logits and returns dhidden (BF16) and dweight
+ * (the head's dtype, rows >= V exactly 0); no [N, V] tensor is ever written.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    row-major and contiguous; the caller allocates and owns every buffer and
+ *    the library allocates no device memory.  Work is enqueued on `stream`
+ *    (a cudaStream_t; NULL = the legacy default stream) and runs
+ *    asynchronously; outputs are valid once the stream has reached that point.
+ *  - hidden:  BF16 [N, H];  weight: [Vp, H], BF16 or FP32 (w_dtype);
+ *    labels: int64 [N], not shifted (labels[n] is the target of hidden[n]).
+ *  - H must be a multiple of 8 (16-byte rows for the tensor-memory-access
+ *    engine); hidden, weight, dhidden, dweight and workspace must be 16-byte
+ *    aligned; labels, loss and lse 8- resp. 4-byte aligned.
+ *  - Arguments are checked on the host before anything is enqueued; a bad
+ *    argument returns an error status and enqueues nothing.  Nothing throws or
+ *    aborts across this boundary.
+ *  - Labels outside [0, V) that are not ignore_index cannot be checked on the
+ *    host without a device read; the kernels treat them as ignored (zero loss,
+ *    zero gradient) and raise FLCE_ERR_BAD_LABEL in a per-device error word
+ *    that flce_get_error() reports and clears.
+ */
+#ifndef FLCE_H_
+#define FLCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* flce_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or option        */
+  FLCE_ERR_WORKSPACE = 2,   /* workspace NULL or smaller than required       */
+  FLCE_ERR_UNSUPPORTED = 3, /* no sm_100a device / too large for this build  */
+  FLCE_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed   */
+  FLCE_ERR_BAD_LABEL = 5,   /* (flce_get_error) a label outside [0,V) seen   */
+  FLCE_ERR_TIMEOUT = 6      /* (flce_get_error) a pipeline wait ran out      */
+} flce_status;
+
+typedef enum { FLCE_SUM = 0, FLCE_MEAN = 1, FLCE_NONE = 2 } flce_reduction;
+typedef enum { FLCE_BF16 = 0, FLCE_F32 = 1 } flce_dtype;
+
+/*
+ * Bytes of workspace that flce_forward and flce_backward want for this shape
+ * (one buffer serves both).  Pure host arithmetic.  Returns 0 for invalid
+ * sizes.  unpadded_vocab <= 0 means padded_vocab.  The backward also accepts a
+ * smaller workspace (down to flce_workspace_min_size) and then streams the
+ * vocabulary in narrower chunks.
+ */
+size_t flce_workspace_size(int64_t n_tokens, int64_t hidden, int64_t padded_vocab,
+                           int64_t unpadded_vocab, int w_dtype);
+size_t flce_workspace_min_size(int64_t n_tokens, int64_t hidden, int64_t padded_vocab,
+                               int64_t unpadded_vocab, int w_dtype);
+
+/*
+ * Forward: the loss and the per-token logsumexp.
+ *   Defines: linear_ce page, FusedLinearCrossEntropy(ignore_index=-100,
+ *   logit_softcapping=0, reduction='sum') and forward(hidden_states, labels,
+ *   lm_weight, num_label_tokens); inkling2 page for unpadded_vocab and the
+ *   BF16/FP32 contract.
+ *   unpadded_vocab   V: rows of the head that enter the softmax; <= 0 means Vp.
+ *   ignore_index     label value that contributes neither loss nor gradient.
+ *   softcap          c >= 0; 0 disables the softcap.
+ *   reduction        FLCE_SUM (default of the pages), FLCE_MEAN or FLCE_NONE.
+ *   num_label_tokens > 0: divide the summed loss by it (FLCE_SUM only);
+ *                    <= 0: no normalisation.
+ *   loss   out, FP32: [1] for SUM/MEAN (MEAN with no valid label gives NaN),
+ *          [N] per-token losses for NONE.
+ *   lse    out, FP32 [N]: per-token logsumexp of the capped logits (all
+ *          tokens, ignored ones included); flce_backward consumes it.
+ *   workspace, ws_bytes: device scratch of at least
+ *          flce_workspace_size(...) bytes; contents are overwritten.
+ * Returns FLCE_OK or an error status.  N == 0 is valid (loss 0, NaN for MEAN).
+ */
+int flce_forward(const void* hidden, const void* weight, int w_dtype, const int64_t* labels,
+                 int64_t n_tokens, int64_t hidden_size, int64_t padded_vocab,
+                 int64_t unpadded_vocab, int64_t ignore_index, float softcap,
+                 int reduction, int64_t num_label_tokens, float* loss, float* lse,
+                 void* workspace, size_t ws_bytes, flce_stream_t stream);
+
+/*
+ * Backward: gradients of the loss above, recomputing the logits.
+ *   Defines: chunked_ce page, _ChunkedCrossEntropySum.backward (recompute the
+ *   FP32 softmax instead of storing it); inkling2 page ("Gradients reach the"
+ *   padded head through the slice and cast: rows >= V get exactly 0).
+ *   Same shape/option arguments as flce_forward.
+ *   grad_loss  in, FP32 device: [1] for SUM/MEAN, [N] for NONE.
+ *   lse        in, FP32 [N]: the lse written by flce_forward on the same inputs.
+ *   dhidden    out, BF16 [N, H] (overwritten).
+ *   dweight    out, [Vp, H] in w_dtype (overwritten; rows [V, Vp) set to 0).
+ *   workspace  >= flce_workspace_min_size(...) bytes; with less than
+ *              flce_workspace_size(...) the vocabulary is processed in
+ *              narrower chunks (same result, more passes over dhidden).
+ * Ignored tokens get exactly-zero dhidden rows and add nothing to dweight.
+ */
+int flce_backward(const void* hidden, const void* weight, int w_dtype, const int64_t* labels,
+                  int64_t n_tokens, int64_t hidden_size, int64_t padded_vocab,
+                  int64_t unpadded_vocab, int64_t ignore_index, float softcap,
+                  int reduction, int64_t num_label_tokens, const float* grad_loss,
+                  const float* lse, void* dhidden, void* dweight,
+                  void* workspace, size_t ws_bytes, flce_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error word:
+ * FLCE_ERR_BAD_LABEL if a kernel saw a label outside [0, V) that was not
+ * ignore_index, FLCE_ERR_TIMEOUT if a pipeline wait gave up (the affected
+ * output is then incomplete), FLCE_ERR_CUDA if the synchronisation failed,
+ * else FLCE_OK.  The word is shared by every call on the device since the
+ * last read.
+ */
+int flce_get_error(flce_stream_t stream);
+
+/* Static description of a status code. */
+const char* flce_status_string(int status);
+
+/* Algorithmic FLOPs of one forward + backward for a shape, for reports:
+ * 8*N*V*H (forward GEMM, recompute GEMM, dW GEMM, dh GEMM; V unpadded). */
+double flce_flops_fwd_bwd(int64_t n_tokens, int64_t hidden_size, int64_t unpadded_vocab);
+
+/*
+ * Self-test of the tensor-core GEMM the path is built on (no counterpart on
+ * the pages; for tests):  D[M, N] (FP32, row-major) = A . B^T over K, with
+ *   A: a_mn == 0 -> BF16 [M, K] (K contiguous); a_mn == 1 -> BF16 [K, M];
+ *   B: b_mn == 0 -> BF16 [N, K];                b_mn == 1 -> BF16 [K, N].
+ * Sizes must be positive, N, K (K-contiguous operands) and M/N (MN-contiguous
+ * operands) multiples of 8.  Device pointers, asynchronous on `stream`.
+ */
+int flce_selftest_gemm(const void* a, const void* b, float* d, int64_t m, int64_t n,
+                       int64_t k, int a_mn, int b_mn, flce_stream_t stream);
+
+/*
+ * Self-test of the bounded pipeline waits (no counterpart on the pages):
+ * launches one block that waits on a barrier nothing ever arrives on, with a
+ * limit of `timeout_us` microseconds (1..2000000).  The kernel gives up, sets
+ * the timeout bit of the error word and returns; the context stays usable.
+ * flce_get_error() then reports FLCE_ERR_TIMEOUT.
+ */
+int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLCE_H_ */

@@ -1,0 +1,267 @@
+// epilogues.cuh - per-tile epilogues of the tensor-core GEMM.  Each runs on
+// one epilogue thread that owns accumulator row `row` (0..127) of tile
+// (mt, nt) and reads its 256 FP32 columns from tensor memory 32 at a time.
+// tcgen05.ld is warp-collective, so rows past the problem edge still load and
+// only skip their stores.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "gemm_sm100.cuh"
+
+namespace flce {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Softcap c*tanh(z/c) from tanh(x) = 1 - 2/(exp(2x) + 1); also returns
+// d(c*tanh(z/c))/dz = 1 - tanh^2 = 4r(1-r) with r = 1/(exp(2x)+1), which stays
+// finite at both ends (r -> 0 and r -> 1).  k = 2*log2(e)/c.
+__device__ __forceinline__ float softcap_value(float z, float c, float k) {
+  const float r = fast_rcp(fast_exp2(z * k) + 1.0f);
+  return c - 2.0f * c * r;
+}
+__device__ __forceinline__ float softcap_value_grad(float z, float c, float k, float& dcap) {
+  const float r = fast_rcp(fast_exp2(z * k) + 1.0f);
+  dcap = 4.0f * r * (1.0f - r);
+  return c - 2.0f * c * r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// -------------------------------------------------------------------------
+// Forward: logits tile -> per-row partial (max, sum of exponentials) over the
+// tile's live vocabulary columns, plus the label's capped logit.
+//   Rows are tokens (A = hidden), columns are head rows (B = W).  Partials are
+//   in base 2: m = max_v zc*log2(e), s = sum_v 2^(zc*log2(e) - m).
+// -------------------------------------------------------------------------
+struct EpiForward {
+  struct Params {
+    const int64_t* labels;
+    int64_t n_tokens;
+    int64_t vocab;        // unpadded V: columns >= V never enter the softmax
+    float softcap;        // 0 = off
+    float softcap_k;      // 2*log2(e)/softcap
+    float* part_m;        // [v_tiles][n_tokens]
+    float* part_s;        // [v_tiles][n_tokens]
+    float* label_logit;   // [n_tokens]: zc at the label (written by the tile holding it)
+  };
+
+  static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
+                                              int row) {
+    const int64_t n = static_cast<int64_t>(mt) * kBM + row;
+    const bool live = n < p.n_tokens;
+    const int64_t vbase = static_cast<int64_t>(nt) * kBN;
+    const int64_t y = live ? p.labels[n] : -1;
+    const int64_t ylocal = y - vbase;
+    const int ncols = static_cast<int>(min(static_cast<int64_t>(kBN), p.vocab - vbase));
+    float m = -INFINITY, s = 0.0f, zl = 0.0f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_load_32cols(taddr + c0, v);
+      if (p.softcap > 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = softcap_value(v[j], p.softcap, p.softcap_k);
+      }
+      if (ylocal >= c0 && ylocal < c0 + 32) {
+        // Pick column ylocal - c0 with a select tree on its bits (no local-memory indexing).
+        const int jl = static_cast<int>(ylocal - c0);
+        float t16[16], t8[8], t4[4], t2[2];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) t16[j] = (jl & 16) ? v[j + 16] : v[j];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t8[j] = (jl & 8) ? t16[j + 8] : t16[j];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) t4[j] = (jl & 4) ? t8[j + 4] : t8[j];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) t2[j] = (jl & 2) ? t4[j + 2] : t4[j];
+        zl = (jl & 1) ? t2[1] : t2[0];
+      }
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float u = (c0 + j < ncols) ? v[j] * kLog2e : -INFINITY;
+        v[j] = u;
+        cmax = fmaxf(cmax, u);
+      }
+      const float mn = fmaxf(m, cmax);
+      if (mn != -INFINITY) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc += fast_exp2(v[j] - mn);
+        s = s * fast_exp2(m - mn) + acc;
+        m = mn;
+      }
+    }
+    if (live) {
+      p.part_m[static_cast<int64_t>(nt) * p.n_tokens + n] = m;
+      p.part_s[static_cast<int64_t>(nt) * p.n_tokens + n] = s;
+      if (ylocal >= 0 && ylocal < ncols) p.label_logit[n] = zl;
+    }
+  }
+};
+
+// -------------------------------------------------------------------------
+// Backward recompute: logits tile -> gradient of the loss w.r.t. the logits,
+//   G[n, v] = s_n * (softmax(zc)[n, v] - [v == y_n]) * dzc/dz,   0 for v >= V,
+// rounded to BF16 and stored to the chunk buffer G[n, v - v0].
+// -------------------------------------------------------------------------
+struct EpiGrad {
+  struct Params {
+    const int64_t* labels;
+    int64_t n_tokens;
+    int64_t vocab;       // unpadded V
+    int64_t v0;          // vocabulary index of GEMM column 0 (chunk start)
+    float softcap;
+    float softcap_k;
+    const float* lse2;   // [n_tokens] logsumexp * log2(e)
+    const float* scale;  // [n_tokens] d loss / d token loss (0 if ignored)
+    __nv_bfloat16* g;    // [n_tokens][ldg]
+    int64_t ldg;
+  };
+
+  static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
+                                              int row) {
+    const int64_t n = static_cast<int64_t>(mt) * kBM + row;
+    const bool live = n < p.n_tokens;
+    const int64_t vbase = p.v0 + static_cast<int64_t>(nt) * kBN;
+    const int64_t y = live ? p.labels[n] : -1;
+    const int64_t ylocal = y - vbase;
+    const float l2 = live ? p.lse2[n] : 0.0f;
+    const float sc = live ? p.scale[n] : 0.0f;
+    const int ncols = static_cast<int>(min(static_cast<int64_t>(kBN), p.vocab - vbase));
+    uint4* out = reinterpret_cast<uint4*>(p.g + (live ? n : 0) * p.ldg + static_cast<int64_t>(nt) * kBN);
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_load_32cols(taddr + c0, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float zc = v[j], dcap = 1.0f;
+        if (p.softcap > 0.0f) zc = softcap_value_grad(v[j], p.softcap, p.softcap_k, dcap);
+        const float prob = fast_exp2(zc * kLog2e - l2);
+        const float onehot = (c0 + j == ylocal) ? 1.0f : 0.0f;
+        const float gr = (prob - onehot) * dcap * sc;
+        v[j] = (c0 + j < ncols) ? gr : 0.0f;
+      }
+      if (live) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+          out[c0 / 8 + q] = w;
+        }
+      }
+    }
+  }
+};
+
+// -------------------------------------------------------------------------
+// Plain store of D rows (dW chunk rows, or the self-test GEMM's output):
+// row r of the tile goes to out[(row0 + r) * ldo + col], as BF16 or FP32.
+// `cols` is a multiple of 8.
+// -------------------------------------------------------------------------
+struct EpiStoreRows {
+  struct Params {
+    void* out;
+    int64_t ldo;
+    int64_t rows;
+    int64_t cols;
+    int f32;
+  };
+
+  static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
+                                              int row) {
+    const int64_t r = static_cast<int64_t>(mt) * kBM + row;
+    const bool live = r < p.rows;
+    const int64_t h0 = static_cast<int64_t>(nt) * kBN;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_load_32cols(taddr + c0, v);
+      if (!live) continue;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t h = h0 + c0 + 8 * q;
+        if (h >= p.cols) break;
+        if (p.f32) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + r * p.ldo + h);
+          o[0] = make_float4(v[8 * q + 0], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]);
+          o[1] = make_float4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]);
+        } else {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + r * p.ldo + h) = w;
+        }
+      }
+    }
+  }
+};
+
+// -------------------------------------------------------------------------
+// dhidden accumulation over vocabulary chunks, exclusive per tile:
+//   mode 0 (first chunk)  acc32  = D
+//   mode 1 (middle)       acc32 += D
+//   mode 2 (last)         out    = bf16(acc32 + D)
+//   mode 3 (only chunk)   out    = bf16(D)
+// -------------------------------------------------------------------------
+struct EpiAccumRows {
+  struct Params {
+    float* acc32;          // [rows][ld]
+    __nv_bfloat16* out;    // [rows][ld]
+    int64_t ld;
+    int64_t rows;
+    int64_t cols;          // multiple of 8
+    int mode;
+  };
+
+  static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
+                                              int row) {
+    const int64_t r = static_cast<int64_t>(mt) * kBM + row;
+    const bool live = r < p.rows;
+    const int64_t h0 = static_cast<int64_t>(nt) * kBN;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_load_32cols(taddr + c0, v);
+      if (!live) continue;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t h = h0 + c0 + 8 * q;
+        if (h >= p.cols) break;
+        float* a = p.acc32 + r * p.ld + h;
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = v[8 * q + i];
+        if (p.mode == 1 || p.mode == 2) {
+          const float4 a0 = reinterpret_cast<const float4*>(a)[0];
+          const float4 a1 = reinterpret_cast<const float4*>(a)[1];
+          x[0] += a0.x; x[1] += a0.y; x[2] += a0.z; x[3] += a0.w;
+          x[4] += a1.x; x[5] += a1.y; x[6] += a1.z; x[7] += a1.w;
+        }
+        if (p.mode <= 1) {
+          reinterpret_cast<float4*>(a)[0] = make_float4(x[0], x[1], x[2], x[3]);
+          reinterpret_cast<float4*>(a)[1] = make_float4(x[4], x[5], x[6], x[7]);
+        } else {
+          uint4 w;
+          w.x = pack_bf16x2(x[0], x[1]);
+          w.y = pack_bf16x2(x[2], x[3]);
+          w.z = pack_bf16x2(x[4], x[5]);
+          w.w = pack_bf16x2(x[6], x[7]);
+          *reinterpret_cast<uint4*>(p.out + r * p.ld + h) = w;
+        }
+      }
+    }
+  }
+};
+
+}  // namespace flce

@@ -1,0 +1,731 @@
+// flce.cu - the C ABI (include/flce.h) of the sm_100a fused LM-head projection
+// + cross-entropy, its auxiliary kernels and the host-side planning.
+//
+// Forward  (nemo_automodel.components.models.inkling2.loss,
+//           Inkling2FusedLinearCrossEntropy: BF16 x BF16 -> FP32, softcap and
+//           CE in FP32, rows >= unpadded_vocab never enter the softmax):
+//   [cast]  FP32 head rows [0, V) -> BF16 (only for an FP32 head)
+//   K1      tensor-core GEMM hidden . W^T, epilogue: softcap, per-tile
+//           (max, sum exp) and the label's logit  -> partials [V/256][N]
+//   K2      merge partials per token -> lse, token loss, block sums
+//   K2b     deterministic final sum -> loss (/ num_label_tokens, or mean)
+// Backward (nemo_automodel.components.loss.chunked_ce,
+//           _ChunkedCrossEntropySum.backward: recompute instead of storing):
+//   prep    per-token gradient scale s_n, lse * log2(e)
+//   per vocabulary chunk [v0, v0 + Vc):
+//     K3    GEMM hidden . W[chunk]^T, epilogue: G = s_n (softmax - onehot) dcap
+//           -> BF16 G[N, Vc] (bounded chunk buffer, never [N, V])
+//     K4    GEMM G^T . hidden  -> dW[chunk] (head dtype)
+//     K5    GEMM G . W[chunk]  -> dhidden, FP32 accumulation across chunks,
+//           BF16 on the last chunk
+//   zero    dW rows [V, Vp)
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "flce.h"
+#include "epilogues.cuh"
+#include "gemm_sm100.cuh"
+
+namespace flce {
+
+__device__ unsigned int g_device_error;  // per-device sticky error word (kDevErr*)
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr int kMergeRows = 32;                         // token rows per merge block
+constexpr int kMergeWarps = 8;
+constexpr int kFinalThreads = 256;
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1024;  // TMA coordinates are int32
+constexpr size_t kAlign = 1024;
+constexpr size_t kChunkBudgetBytes = size_t(256) << 20;  // default G chunk buffer
+constexpr int64_t kMinChunk = 4096;
+
+// ------------------------------------------------------------------ kernels
+
+// FP32 -> BF16 (round to nearest even), 8 elements per step.
+__global__ void cast_f32_to_bf16_kernel(const float4* __restrict__ src, uint4* __restrict__ dst,
+                                        int64_t n8) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float4 a = src[2 * i], b = src[2 * i + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x, a.y);
+    w.y = pack_bf16x2(a.z, a.w);
+    w.z = pack_bf16x2(b.x, b.y);
+    w.w = pack_bf16x2(b.z, b.w);
+    dst[i] = w;
+  }
+}
+
+__global__ void zero16_kernel(uint4* __restrict__ dst, int64_t n16) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n16;
+       i += int64_t(gridDim.x) * blockDim.x)
+    dst[i] = make_uint4(0, 0, 0, 0);
+}
+
+// K2: merge the per-tile partials of 32 token rows (8 warps split the tiles),
+// then per token: lse, token loss, label check; per block: loss and count sums.
+__global__ void __launch_bounds__(kMergeRows* kMergeWarps)
+    lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
+                     int v_tiles, int64_t n_tokens, const float* __restrict__ label_logit,
+                     const int64_t* __restrict__ labels, int64_t vocab, int64_t ignore_index,
+                     float* __restrict__ lse_out, float* __restrict__ token_loss,
+                     double* __restrict__ blk_loss, int* __restrict__ blk_cnt,
+                     unsigned* __restrict__ err) {
+  __shared__ float sm_m[kMergeWarps][kMergeRows];
+  __shared__ float sm_s[kMergeWarps][kMergeRows];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t n = int64_t(blockIdx.x) * kMergeRows + lane;
+  float M = -INFINITY, S = 0.0f;
+  if (n < n_tokens) {
+    for (int t = warp; t < v_tiles; t += kMergeWarps) {
+      const float m = part_m[int64_t(t) * n_tokens + n];
+      const float s = part_s[int64_t(t) * n_tokens + n];
+      const float mn = fmaxf(M, m);
+      S = S * exp2f(M - mn) + s * exp2f(m - mn);
+      M = mn;
+    }
+  }
+  sm_m[warp][lane] = M;
+  sm_s[warp][lane] = S;
+  __syncthreads();
+  if (warp != 0) return;
+  float Mt = -INFINITY, St = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) {
+    const float m = sm_m[w][lane], s = sm_s[w][lane];
+    if (m == -INFINITY) continue;
+    const float mn = fmaxf(Mt, m);
+    St = St * exp2f(Mt - mn) + s * exp2f(m - mn);
+    Mt = mn;
+  }
+  double loss = 0.0;
+  int cnt = 0;
+  if (n < n_tokens) {
+    const float lse = (Mt + log2f(St)) * 0.6931471805599453f;
+    const int64_t y = labels[n];
+    bool valid = y != ignore_index;
+    if (valid && (y < 0 || y >= vocab)) {
+      atomicOr(err, kDevErrBadLabel);
+      valid = false;
+    }
+    const float l = valid ? lse - label_logit[n] : 0.0f;
+    lse_out[n] = lse;
+    if (token_loss) token_loss[n] = l;
+    loss = l;
+    cnt = valid ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    loss += __shfl_down_sync(0xffffffffu, loss, o);
+    cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  }
+  if (lane == 0) {
+    blk_loss[blockIdx.x] = loss;
+    blk_cnt[blockIdx.x] = cnt;
+  }
+}
+
+// K2b: fixed-order sum of the block partials -> loss[0].
+__global__ void __launch_bounds__(kFinalThreads)
+    loss_finalize_kernel(const double* __restrict__ blk_loss, const int* __restrict__ blk_cnt,
+                         int nblk, int reduction, int64_t num_label_tokens,
+                         float* __restrict__ loss) {
+  __shared__ double sl[kFinalThreads];
+  __shared__ long long sc[kFinalThreads];
+  double l = 0.0;
+  long long c = 0;
+  for (int i = threadIdx.x; i < nblk; i += kFinalThreads) {
+    l += blk_loss[i];
+    c += blk_cnt[i];
+  }
+  sl[threadIdx.x] = l;
+  sc[threadIdx.x] = c;
+  __syncthreads();
+  for (int s = kFinalThreads / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) {
+      sl[threadIdx.x] += sl[threadIdx.x + s];
+      sc[threadIdx.x] += sc[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    double total = sl[0];
+    if (reduction == FLCE_SUM) {
+      if (num_label_tokens > 0) total /= double(num_label_tokens);
+    } else if (reduction == FLCE_MEAN) {
+      total = sc[0] > 0 ? total / double(sc[0]) : double(NAN);
+    }
+    loss[0] = float(total);
+  }
+}
+
+// Backward prep (one block): valid-label count, per-token gradient scale
+// s_n = d loss / d token loss (0 for ignored / invalid labels), lse * log2(e).
+__global__ void __launch_bounds__(1024)
+    bwd_prep_kernel(const int64_t* __restrict__ labels, int64_t n_tokens, int64_t vocab,
+                    int64_t ignore_index, int reduction, int64_t num_label_tokens,
+                    const float* __restrict__ grad_loss, const float* __restrict__ lse,
+                    float* __restrict__ lse2, float* __restrict__ scale,
+                    unsigned* __restrict__ err) {
+  __shared__ int warp_cnt[32];
+  int cnt = 0;
+  bool bad = false;
+  for (int64_t n = threadIdx.x; n < n_tokens; n += blockDim.x) {
+    const int64_t y = labels[n];
+    if (y == ignore_index) continue;
+    if (y < 0 || y >= vocab) {
+      bad = true;
+      continue;
+    }
+    ++cnt;
+  }
+  if (bad) atomicOr(err, kDevErrBadLabel);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  int total = 0;
+  for (int w = 0; w < int(blockDim.x >> 5); ++w) total += warp_cnt[w];
+  float base = 0.0f;
+  if (reduction == FLCE_SUM) {
+    base = grad_loss[0];
+    if (num_label_tokens > 0) base = float(double(base) / double(num_label_tokens));
+  } else if (reduction == FLCE_MEAN) {
+    base = total > 0 ? float(double(grad_loss[0]) / double(total)) : 0.0f;
+  }
+  for (int64_t n = threadIdx.x; n < n_tokens; n += blockDim.x) {
+    const int64_t y = labels[n];
+    const bool valid = y != ignore_index && y >= 0 && y < vocab;
+    const float g = reduction == FLCE_NONE ? grad_loss[n] : base;
+    scale[n] = valid ? g : 0.0f;
+    lse2[n] = lse[n] * kLog2e;
+  }
+}
+
+// A wait on a barrier that nothing arrives on: exercises the bounded-wait path.
+__global__ void wait_timeout_selftest_kernel(unsigned* err, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ PipeCtl ctl;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    GemmShape g{};
+    g.err = err;
+    g.timeout_ns = timeout_ns;
+    wait_phase(smem_u32(&bar), 0, &ctl, g);
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ host side
+
+struct DeviceInfo {
+  bool init = false;
+  int status = FLCE_OK;
+  int num_sms = 0;
+  unsigned* err = nullptr;
+};
+
+static std::mutex g_mutex;
+static DeviceInfo g_dev[64];
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FLCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    d.init = true;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.status = FLCE_ERR_CUDA;
+    } else if (major != 10 || minor != 0) {
+      d.status = FLCE_ERR_UNSUPPORTED;  // built for sm_100a only
+    } else if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error) !=
+               cudaSuccess) {
+      d.status = FLCE_ERR_CUDA;
+    }
+    if (d.status == FLCE_OK && g_encode == nullptr) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        d.status = FLCE_ERR_CUDA;
+      else
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  if (d.status != FLCE_OK) {
+    d.init = false;  // retry next call (e.g. after the caller fixed the device)
+    return d.status;
+  }
+  *out = &d;
+  return FLCE_OK;
+}
+
+// 2-D BF16 tensor map, 128-byte swizzle, zero fill outside [inner, outer).
+static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// K-major operand [outer rows][inner K]: one box of 64 K x `rows` rows.
+static bool tmap_kmajor(CUtensorMap* tm, const void* base, int64_t k, int64_t rows,
+                        int64_t ld_elems, int box_rows) {
+  return make_tmap(tm, base, uint64_t(k), uint64_t(rows), uint64_t(ld_elems) * 2, 64,
+                   uint32_t(box_rows));
+}
+// MN-major operand [outer K rows][inner MN]: boxes of 64 MN x 64 K.
+static bool tmap_mnmajor(CUtensorMap* tm, const void* base, int64_t mn, int64_t k,
+                         int64_t ld_elems) {
+  return make_tmap(tm, base, uint64_t(mn), uint64_t(k), uint64_t(ld_elems) * 2, 64, 64);
+}
+
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
+  TileRaster r;
+  r.m_tiles = int(cdiv(m, kBM));
+  r.n_tiles = int(cdiv(n, kBN));
+  // Keep the group's A panel (group_m x 128 rows x K) around 48 MB so it stays in L2.
+  const int64_t panel = int64_t(kBM) * std::max<int64_t>(k, 1) * 2;
+  int64_t gm = std::max<int64_t>(1, (int64_t(48) << 20) / panel);
+  r.group_m = int(std::min<int64_t>(gm, r.m_tiles));
+  return r;
+}
+
+template <class Epi, bool kAMn, bool kBMn>
+static int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmShape g,
+                       const typename Epi::Params& ep, const DeviceInfo& dev, cudaStream_t st) {
+  g.raster = make_raster(g.m, g.n, g.k);
+  g.tiles = int64_t(g.raster.m_tiles) * g.raster.n_tiles;
+  g.err = dev.err;
+  g.timeout_ns = kDefaultTimeoutNs;
+  if (g.tiles == 0) return FLCE_OK;
+  auto kern = tc_gemm_kernel<Epi, kAMn, kBMn>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(kGemmSmemBytes)) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  const int grid = int(std::min<int64_t>(dev.num_sms, g.tiles));
+  kern<<<grid, kThreads, kGemmSmemBytes, st>>>(ta, tb, g, ep);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+static int launch_zero(void* p, size_t bytes, const DeviceInfo& dev, cudaStream_t st) {
+  if (bytes == 0) return FLCE_OK;
+  const int64_t n16 = int64_t(bytes / 16);
+  const int grid = int(std::min<int64_t>(int64_t(dev.num_sms) * 8, cdiv(n16, 256)));
+  zero16_kernel<<<std::max(grid, 1), 256, 0, st>>>(static_cast<uint4*>(p), n16);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+static int launch_cast(const float* src, __nv_bfloat16* dst, int64_t elems,
+                       const DeviceInfo& dev, cudaStream_t st) {
+  const int64_t n8 = elems / 8;
+  if (n8 == 0) return FLCE_OK;
+  const int grid = int(std::min<int64_t>(int64_t(dev.num_sms) * 8, cdiv(n8, 256)));
+  cast_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
+                                                reinterpret_cast<uint4*>(dst), n8);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- planning
+
+struct Shape {
+  int64_t n, h, vp, v;
+  int w_dtype;
+};
+
+struct FwdPlan {
+  int64_t v_tiles, nblk;
+  size_t off_pm, off_ps, off_zl, off_bl, off_bc, off_wb, total;
+};
+
+struct BwdPlan {
+  int64_t vc;  // vocabulary chunk width (multiple of 256)
+  size_t off_lse2, off_scale, off_dh32, off_wb, off_g, fixed, total;
+};
+
+static FwdPlan plan_forward(const Shape& s) {
+  FwdPlan p{};
+  p.v_tiles = cdiv(s.v, kBN);
+  p.nblk = cdiv(s.n, kMergeRows);
+  size_t o = 0;
+  p.off_pm = o;  o = align_up(o + size_t(p.v_tiles) * s.n * 4);
+  p.off_ps = o;  o = align_up(o + size_t(p.v_tiles) * s.n * 4);
+  p.off_zl = o;  o = align_up(o + size_t(s.n) * 4);
+  p.off_bl = o;  o = align_up(o + size_t(p.nblk) * 8);
+  p.off_bc = o;  o = align_up(o + size_t(p.nblk) * 4);
+  p.off_wb = o;  o = align_up(o + (s.w_dtype == FLCE_F32 ? size_t(s.v) * s.h * 2 : 0));
+  p.total = std::max(o, kAlign);  // never zero, so N = 0 still has a valid buffer
+  return p;
+}
+
+static int64_t default_chunk(const Shape& s) {
+  const int64_t cap = cdiv(cdiv(s.v, 4), kBN) * kBN;  // at most a quarter of the vocabulary
+  int64_t budget = int64_t(kChunkBudgetBytes / (2 * size_t(std::max<int64_t>(s.n, 1))));
+  budget = budget / kBN * kBN;
+  return std::max<int64_t>(kBN, std::min(cap, std::max(kMinChunk, budget)));
+}
+
+static BwdPlan plan_backward(const Shape& s, int64_t vc) {
+  BwdPlan p{};
+  p.vc = vc;
+  size_t o = 0;
+  p.off_lse2 = o;  o = align_up(o + size_t(s.n) * 4);
+  p.off_scale = o; o = align_up(o + size_t(s.n) * 4);
+  p.off_dh32 = o;  o = align_up(o + size_t(s.n) * s.h * 4);
+  p.off_wb = o;    o = align_up(o + (s.w_dtype == FLCE_F32 ? size_t(s.v) * s.h * 2 : 0));
+  p.fixed = o;
+  p.off_g = o;     o = align_up(o + size_t(s.n) * vc * 2);
+  p.total = o;
+  return p;
+}
+
+static bool shape_ok(int64_t n, int64_t h, int64_t vp, int64_t v, int w_dtype) {
+  if (n < 0 || h <= 0 || vp <= 0) return false;
+  if (h % 8 != 0) return false;
+  if (v <= 0 || v > vp) return false;
+  if (n > kMaxDim || h > kMaxDim || vp > kMaxDim) return false;
+  if (w_dtype != FLCE_BF16 && w_dtype != FLCE_F32) return false;
+  return true;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static int check_common(const void* hidden, const void* weight, int w_dtype,
+                        const int64_t* labels, int64_t n, int64_t h, int64_t vp, int64_t v,
+                        float softcap, int reduction, int64_t num_label_tokens) {
+  if (!shape_ok(n, h, vp, v, w_dtype)) return FLCE_ERR_INVALID_ARG;
+  if (!(softcap >= 0.0f) || !std::isfinite(softcap)) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_SUM && reduction != FLCE_MEAN && reduction != FLCE_NONE)
+    return FLCE_ERR_INVALID_ARG;
+  if (num_label_tokens > 0 && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  if (weight == nullptr || !aligned(weight, 16)) return FLCE_ERR_INVALID_ARG;
+  if (n > 0) {
+    if (hidden == nullptr || labels == nullptr) return FLCE_ERR_INVALID_ARG;
+    if (!aligned(hidden, 16) || !aligned(labels, 8)) return FLCE_ERR_INVALID_ARG;
+  }
+  return FLCE_OK;
+}
+
+}  // namespace flce
+
+using namespace flce;
+
+// ====================================================================== C ABI
+
+extern "C" size_t flce_workspace_size(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
+                                      int w_dtype) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  if (!shape_ok(n, h, vp, v, w_dtype)) return 0;
+  const Shape s{n, h, vp, v, w_dtype};
+  return std::max(plan_forward(s).total, plan_backward(s, default_chunk(s)).total);
+}
+
+extern "C" size_t flce_workspace_min_size(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
+                                          int w_dtype) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  if (!shape_ok(n, h, vp, v, w_dtype)) return 0;
+  const Shape s{n, h, vp, v, w_dtype};
+  return std::max(plan_forward(s).total, plan_backward(s, kBN).total);
+}
+
+extern "C" double flce_flops_fwd_bwd(int64_t n, int64_t h, int64_t v) {
+  return 8.0 * double(n) * double(v) * double(h);
+}
+
+extern "C" const char* flce_status_string(int status) {
+  switch (status) {
+    case FLCE_OK: return "ok";
+    case FLCE_ERR_INVALID_ARG: return "invalid argument";
+    case FLCE_ERR_WORKSPACE: return "workspace missing or too small";
+    case FLCE_ERR_UNSUPPORTED: return "unsupported device or size (needs sm_100)";
+    case FLCE_ERR_CUDA: return "CUDA runtime error";
+    case FLCE_ERR_BAD_LABEL: return "label outside [0, unpadded_vocab) that is not ignore_index";
+    case FLCE_ERR_TIMEOUT: return "a pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
+                            const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                            int64_t unpadded, int64_t ignore_index, float softcap, int reduction,
+                            int64_t num_label_tokens, float* loss, float* lse, void* workspace,
+                            size_t ws_bytes, flce_stream_t stream) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
+                        num_label_tokens);
+  if (st != FLCE_OK) return st;
+  if ((n > 0 || reduction != FLCE_NONE) && (loss == nullptr || !aligned(loss, 4)))
+    return FLCE_ERR_INVALID_ARG;
+  if (n > 0 && (lse == nullptr || !aligned(lse, 4))) return FLCE_ERR_INVALID_ARG;
+  const Shape s{n, h, vp, v, w_dtype};
+  const FwdPlan p = plan_forward(s);
+  if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p.total)
+    return FLCE_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* blk_loss = reinterpret_cast<double*>(ws + p.off_bl);
+  int* blk_cnt = reinterpret_cast<int*>(ws + p.off_bc);
+
+  if (n == 0) {
+    if (reduction == FLCE_NONE) return FLCE_OK;
+    loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(blk_loss, blk_cnt, 0, reduction,
+                                                      num_label_tokens, loss);
+    return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  }
+
+  const void* wb = weight;
+  if (w_dtype == FLCE_F32) {
+    wb = ws + p.off_wb;
+    if ((st = launch_cast(static_cast<const float*>(weight),
+                          reinterpret_cast<__nv_bfloat16*>(ws + p.off_wb), v * h, *dev, cs)) !=
+        FLCE_OK)
+      return st;
+  }
+
+  CUtensorMap ta, tb;
+  if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBN))
+    return FLCE_ERR_CUDA;
+  GemmShape g{};
+  g.m = n;
+  g.n = v;
+  g.k = h;
+  EpiForward::Params ep{};
+  ep.labels = labels;
+  ep.n_tokens = n;
+  ep.vocab = v;
+  ep.softcap = softcap;
+  ep.softcap_k = softcap > 0.0f ? 2.0f * kLog2e / softcap : 0.0f;
+  ep.part_m = reinterpret_cast<float*>(ws + p.off_pm);
+  ep.part_s = reinterpret_cast<float*>(ws + p.off_ps);
+  ep.label_logit = reinterpret_cast<float*>(ws + p.off_zl);
+  if ((st = launch_gemm<EpiForward, false, false>(ta, tb, g, ep, *dev, cs)) != FLCE_OK) return st;
+
+  lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
+      ep.part_m, ep.part_s, int(p.v_tiles), n, ep.label_logit, labels, v, ignore_index, lse,
+      reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (reduction != FLCE_NONE) {
+    loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(blk_loss, blk_cnt, int(p.nblk), reduction,
+                                                      num_label_tokens, loss);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  return FLCE_OK;
+}
+
+extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype,
+                             const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                             int64_t unpadded, int64_t ignore_index, float softcap,
+                             int reduction, int64_t num_label_tokens, const float* grad_loss,
+                             const float* lse, void* dhidden, void* dweight, void* workspace,
+                             size_t ws_bytes, flce_stream_t stream) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
+                        num_label_tokens);
+  if (st != FLCE_OK) return st;
+  if (dweight == nullptr || !aligned(dweight, 16)) return FLCE_ERR_INVALID_ARG;
+  if (n > 0) {
+    if (grad_loss == nullptr || lse == nullptr || dhidden == nullptr) return FLCE_ERR_INVALID_ARG;
+    if (!aligned(grad_loss, 4) || !aligned(lse, 4) || !aligned(dhidden, 16))
+      return FLCE_ERR_INVALID_ARG;
+  }
+  const Shape s{n, h, vp, v, w_dtype};
+  const BwdPlan p0 = plan_backward(s, kBN);
+  if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p0.total)
+    return FLCE_ERR_WORKSPACE;
+  // Widest chunk that fits the workspace, up to the default.
+  int64_t vc = default_chunk(s);
+  if (n > 0) {
+    const int64_t fit = int64_t((ws_bytes - p0.fixed) / (2 * size_t(n))) / kBN * kBN;
+    vc = std::max<int64_t>(kBN, std::min(vc, fit));
+  }
+  const BwdPlan p = plan_backward(s, vc);
+  if (ws_bytes < p.total) return FLCE_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t wsz = w_dtype == FLCE_F32 ? 4 : 2;
+
+  // Rows the softmax never sees get exactly zero gradient; with no tokens, all rows.
+  const int64_t zero_from = n == 0 ? 0 : v;
+  if ((st = launch_zero(static_cast<uint8_t*>(dweight) + size_t(zero_from) * h * wsz,
+                        size_t(vp - zero_from) * h * wsz, *dev, cs)) != FLCE_OK)
+    return st;
+  if (n == 0) return FLCE_OK;
+
+  const void* wb = weight;
+  if (w_dtype == FLCE_F32) {
+    wb = ws + p.off_wb;
+    if ((st = launch_cast(static_cast<const float*>(weight),
+                          reinterpret_cast<__nv_bfloat16*>(ws + p.off_wb), v * h, *dev, cs)) !=
+        FLCE_OK)
+      return st;
+  }
+  float* lse2 = reinterpret_cast<float*>(ws + p.off_lse2);
+  float* scale = reinterpret_cast<float*>(ws + p.off_scale);
+  float* dh32 = reinterpret_cast<float*>(ws + p.off_dh32);
+  __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ws + p.off_g);
+  bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, n, v, ignore_index, reduction, num_label_tokens,
+                                      grad_loss, lse, lse2, scale, dev->err);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+
+  CUtensorMap t_hid_k, t_w_k, t_hid_mn, t_w_mn;
+  if (!tmap_kmajor(&t_hid_k, hidden, h, n, h, kBM) || !tmap_kmajor(&t_w_k, wb, h, v, h, kBN) ||
+      !tmap_mnmajor(&t_hid_mn, hidden, h, n, h) || !tmap_mnmajor(&t_w_mn, wb, h, v, h))
+    return FLCE_ERR_CUDA;
+
+  const int64_t chunks = cdiv(v, vc);
+  for (int64_t c = 0; c < chunks; ++c) {
+    const int64_t v0 = c * vc;
+    const int64_t width = std::min(vc, v - v0);
+    const int64_t gcols = cdiv(width, kBN) * kBN;
+
+    // K3: recompute logits for the chunk and form G (BF16) in the chunk buffer.
+    {
+      GemmShape g{};
+      g.m = n;
+      g.n = width;
+      g.k = h;
+      g.b_mn_off = int(v0);
+      EpiGrad::Params ep{};
+      ep.labels = labels;
+      ep.n_tokens = n;
+      ep.vocab = v;
+      ep.v0 = v0;
+      ep.softcap = softcap;
+      ep.softcap_k = softcap > 0.0f ? 2.0f * kLog2e / softcap : 0.0f;
+      ep.lse2 = lse2;
+      ep.scale = scale;
+      ep.g = gbuf;
+      ep.ldg = vc;
+      if ((st = launch_gemm<EpiGrad, false, false>(t_hid_k, t_w_k, g, ep, *dev, cs)) != FLCE_OK)
+        return st;
+    }
+    CUtensorMap t_g_mn, t_g_k;
+    if (!tmap_mnmajor(&t_g_mn, gbuf, gcols, n, vc) || !tmap_kmajor(&t_g_k, gbuf, gcols, n, vc, kBM))
+      return FLCE_ERR_CUDA;
+    // K4: dW[v0 : v0 + width] = G^T . hidden  (contraction over tokens).
+    {
+      GemmShape g{};
+      g.m = width;
+      g.n = h;
+      g.k = n;
+      EpiStoreRows::Params ep{};
+      ep.out = static_cast<uint8_t*>(dweight) + size_t(v0) * h * wsz;
+      ep.ldo = h;
+      ep.rows = width;
+      ep.cols = h;
+      ep.f32 = w_dtype == FLCE_F32;
+      if ((st = launch_gemm<EpiStoreRows, true, true>(t_g_mn, t_hid_mn, g, ep, *dev, cs)) !=
+          FLCE_OK)
+        return st;
+    }
+    // K5: dhidden (+)= G . W[v0 : v0 + width]  (contraction over the chunk).
+    {
+      GemmShape g{};
+      g.m = n;
+      g.n = h;
+      g.k = gcols;
+      g.b_k_off = int(v0);
+      EpiAccumRows::Params ep{};
+      ep.acc32 = dh32;
+      ep.out = static_cast<__nv_bfloat16*>(dhidden);
+      ep.ld = h;
+      ep.rows = n;
+      ep.cols = h;
+      ep.mode = chunks == 1 ? 3 : (c == 0 ? 0 : (c == chunks - 1 ? 2 : 1));
+      if ((st = launch_gemm<EpiAccumRows, false, true>(t_g_k, t_w_mn, g, ep, *dev, cs)) !=
+          FLCE_OK)
+        return st;
+    }
+  }
+  return FLCE_OK;
+}
+
+extern "C" int flce_get_error(flce_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int st = device_info(&dev);
+  if (st != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  unsigned host = 0;
+  if (cudaMemcpyAsync(&host, dev->err, sizeof(unsigned), cudaMemcpyDeviceToHost, cs) !=
+          cudaSuccess ||
+      cudaMemsetAsync(dev->err, 0, sizeof(unsigned), cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (host & kDevErrTimeout) return FLCE_ERR_TIMEOUT;
+  if (host & kDevErrBadLabel) return FLCE_ERR_BAD_LABEL;
+  return FLCE_OK;
+}
+
+extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_t m, int64_t n,
+                                  int64_t k, int a_mn, int b_mn, flce_stream_t stream) {
+  if (a == nullptr || b == nullptr || d == nullptr || m <= 0 || n <= 0 || k <= 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (m > kMaxDim || n > kMaxDim || k > kMaxDim) return FLCE_ERR_INVALID_ARG;
+  if (n % 8 != 0 || (a_mn ? m % 8 : k % 8) != 0 || (b_mn ? n % 8 : k % 8) != 0)
+    return FLCE_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16)) return FLCE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_info(&dev);
+  if (st != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  CUtensorMap ta, tb;
+  const bool ok_a = a_mn ? tmap_mnmajor(&ta, a, m, k, m) : tmap_kmajor(&ta, a, k, m, k, kBM);
+  const bool ok_b = b_mn ? tmap_mnmajor(&tb, b, n, k, n) : tmap_kmajor(&tb, b, k, n, k, kBN);
+  if (!ok_a || !ok_b) return FLCE_ERR_CUDA;
+  GemmShape g{};
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  EpiStoreRows::Params ep{};
+  ep.out = d;
+  ep.ldo = n;
+  ep.rows = m;
+  ep.cols = n;
+  ep.f32 = 1;
+  if (!a_mn && !b_mn) return launch_gemm<EpiStoreRows, false, false>(ta, tb, g, ep, *dev, cs);
+  if (!a_mn && b_mn) return launch_gemm<EpiStoreRows, false, true>(ta, tb, g, ep, *dev, cs);
+  if (a_mn && !b_mn) return launch_gemm<EpiStoreRows, true, false>(ta, tb, g, ep, *dev, cs);
+  return launch_gemm<EpiStoreRows, true, true>(ta, tb, g, ep, *dev, cs);
+}
+
+extern "C" int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream) {
+  if (timeout_us == 0 || timeout_us > 2000000u) return FLCE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_info(&dev);
+  if (st != FLCE_OK) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      dev->err, uint64_t(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}

@@ -1,0 +1,240 @@
+"""Python binding of libflce.so: argument marshalling only.
+
+Every step of the loss and its gradient runs in the library's CUDA kernels;
+this module checks tensors, allocates outputs and workspace with PyTorch (the
+caller's device memory) and passes raw pointers and the current CUDA stream
+through ctypes.  If the library is missing it raises: there is no fallback.
+
+Entry points mirror include/flce.h:
+  forward(hidden, weight, labels, ...)            -> (loss, lse)
+  backward(hidden, weight, labels, lse, grad, ...) -> (dhidden, dweight)
+  fused_linear_cross_entropy(...)                  autograd-aware convenience
+with the options of the NeMo-AutoModel loss pages
+("nemo_automodel.components.loss.linear_ce", FusedLinearCrossEntropy:
+ignore_index=-100, logit_softcapping=0, reduction='sum', num_label_tokens;
+"nemo_automodel.components.models.inkling2.loss": unpadded_vocab_size and an
+FP32 head rounded to BF16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB_PATH
+
+FLCE_OK = 0
+FLCE_ERR_BAD_LABEL = 5
+FLCE_ERR_TIMEOUT = 6
+STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_INVALID_ARG", 2: "FLCE_ERR_WORKSPACE",
+          3: "FLCE_ERR_UNSUPPORTED", 4: "FLCE_ERR_CUDA", 5: "FLCE_ERR_BAD_LABEL",
+          6: "FLCE_ERR_TIMEOUT"}
+REDUCTIONS = {"sum": 0, "mean": 1, "none": 2}
+W_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+
+_c_i64 = ctypes.c_int64
+_c_int = ctypes.c_int
+_c_ptr = ctypes.c_void_p
+_c_size = ctypes.c_size_t
+
+# name -> (restype, argtypes); the exported C ABI of include/flce.h
+SIGNATURES = {
+    "flce_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int]),
+    "flce_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int]),
+    "flce_forward": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
+                              _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr,
+                              _c_size, _c_ptr]),
+    "flce_backward": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
+                               _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr,
+                               _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "flce_get_error": (_c_int, [_c_ptr]),
+    "flce_status_string": (ctypes.c_char_p, [_c_int]),
+    "flce_flops_fwd_bwd": (ctypes.c_double, [_c_i64, _c_i64, _c_i64]),
+    "flce_selftest_gemm": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_int,
+                                    _c_int, _c_ptr]),
+    "flce_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _c_ptr]),
+}
+
+_LIB = None
+
+
+class FlceError(RuntimeError):
+    def __init__(self, where: str, status: int):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libflce.so (built in-tree).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m lm_head_projection_flce_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _check(where: str, status: int) -> None:
+    if status != FLCE_OK:
+        raise FlceError(where, status)
+
+
+def _stream_handle(device: torch.device, stream=None):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() > 0 else 0)
+
+
+def _vocab(weight: torch.Tensor, unpadded_vocab: int | None) -> int:
+    return weight.shape[0] if unpadded_vocab is None or unpadded_vocab <= 0 else int(unpadded_vocab)
+
+
+def workspace_size(n_tokens: int, hidden: int, padded_vocab: int, unpadded_vocab: int | None,
+                   w_dtype: torch.dtype = torch.bfloat16, minimum: bool = False) -> int:
+    lib = load_library()
+    fn = lib.flce_workspace_min_size if minimum else lib.flce_workspace_size
+    return int(fn(n_tokens, hidden, padded_vocab, unpadded_vocab or 0, W_DTYPES[w_dtype]))
+
+
+def _prepare(hidden, weight, labels):
+    if hidden.dtype != torch.bfloat16:
+        raise TypeError("hidden must be bf16")
+    if weight.dtype not in W_DTYPES:
+        raise TypeError("weight must be bf16 or fp32")
+    if labels.dtype != torch.int64:
+        raise TypeError("labels must be int64")
+    h = hidden.shape[-1]
+    hid = hidden.reshape(-1, h)
+    lab = labels.reshape(-1)
+    if hid.shape[0] != lab.shape[0]:
+        raise ValueError("hidden and labels disagree on the number of tokens")
+    if weight.dim() != 2 or weight.shape[1] != h:
+        raise ValueError("weight must be [vocab, hidden]")
+    for t in (hid, weight, lab):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if t.device != hid.device or t.device.type != "cuda":
+            raise ValueError("tensors must be on one CUDA device")
+    return hid, lab
+
+
+def _workspace(ws, need: int, device) -> torch.Tensor:
+    if ws is None:
+        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    return ws
+
+
+def forward(hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
+            unpadded_vocab: int | None = None, reduction: str = "sum",
+            num_label_tokens: int | None = None, workspace: torch.Tensor | None = None,
+            loss: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Fused projection + cross entropy.  Returns ``(loss, lse)`` (FP32)."""
+    lib = load_library()
+    hid, lab = _prepare(hidden, weight, labels)
+    n, h = hid.shape
+    vp = weight.shape[0]
+    v = _vocab(weight, unpadded_vocab)
+    dev = hid.device
+    red = REDUCTIONS[reduction]
+    if loss is None:
+        loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
+    st = lib.flce_forward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
+                          v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
+                          _ptr(loss), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(dev, stream))
+    _check("flce_forward", st)
+    return (loss if reduction == "none" else loss.reshape(())), lse
+
+
+def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100,
+             softcap: float = 0.0, unpadded_vocab: int | None = None, reduction: str = "sum",
+             num_label_tokens: int | None = None, workspace: torch.Tensor | None = None,
+             dhidden: torch.Tensor | None = None, dweight: torch.Tensor | None = None,
+             stream=None):
+    """Gradients ``(dhidden [.., H] bf16, dweight [Vp, H] in the head's dtype)``."""
+    lib = load_library()
+    hid, lab = _prepare(hidden, weight, labels)
+    n, h = hid.shape
+    vp = weight.shape[0]
+    v = _vocab(weight, unpadded_vocab)
+    dev = hid.device
+    red = REDUCTIONS[reduction]
+    grad = grad_loss.reshape(-1).to(device=dev, dtype=torch.float32).contiguous()
+    if dhidden is None:
+        dhidden = torch.empty_like(hid)
+    if dweight is None:
+        dweight = torch.empty_like(weight)
+    ws = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
+    st = lib.flce_backward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
+                           v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
+                           _ptr(grad), _ptr(lse), _ptr(dhidden), _ptr(dweight), _ptr(ws),
+                           ws.numel(), _stream_handle(dev, stream))
+    _check("flce_backward", st)
+    return dhidden.reshape(hidden.shape), dweight
+
+
+def get_error(device=None, stream=None) -> int:
+    """Synchronise and read-and-clear the device error word (FLCE_* status)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib.flce_get_error(_stream_handle(dev, stream)))
+
+
+def selftest_gemm(a, b, m: int, n: int, k: int, a_mn: bool, b_mn: bool) -> torch.Tensor:
+    """D = A . B^T through the library's tensor-core GEMM (tests only)."""
+    lib = load_library()
+    d = torch.empty(m, n, dtype=torch.float32, device=a.device)
+    st = lib.flce_selftest_gemm(_ptr(a), _ptr(b), _ptr(d), m, n, k, int(a_mn), int(b_mn),
+                                _stream_handle(a.device))
+    _check("flce_selftest_gemm", st)
+    return d
+
+
+def selftest_wait_timeout(timeout_us: int, device=None) -> None:
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check("flce_selftest_wait_timeout",
+           lib.flce_selftest_wait_timeout(timeout_us, _stream_handle(dev)))
+
+
+class _FusedLinearCE(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, hidden, weight, labels, ignore_index, softcap, unpadded_vocab, reduction,
+                num_label_tokens):
+        loss, lse = forward(hidden, weight, labels, ignore_index=ignore_index, softcap=softcap,
+                            unpadded_vocab=unpadded_vocab, reduction=reduction,
+                            num_label_tokens=num_label_tokens)
+        ctx.save_for_backward(hidden, weight, labels, lse)
+        ctx.opts = (ignore_index, softcap, unpadded_vocab, reduction, num_label_tokens)
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        hidden, weight, labels, lse = ctx.saved_tensors
+        ii, c, uv, red, nlt = ctx.opts
+        dh, dw = backward(hidden, weight, labels, lse, grad_out, ignore_index=ii, softcap=c,
+                          unpadded_vocab=uv, reduction=red, num_label_tokens=nlt)
+        return dh, dw, None, None, None, None, None, None
+
+
+def fused_linear_cross_entropy(hidden, weight, labels, *, ignore_index: int = -100,
+                               softcap: float = 0.0, unpadded_vocab: int | None = None,
+                               reduction: str = "sum", num_label_tokens: int | None = None):
+    """Autograd-aware loss: gradients flow to ``hidden`` and ``weight``."""
+    return _FusedLinearCE.apply(hidden, weight, labels, ignore_index, softcap, unpadded_vocab,
+                                reduction, num_label_tokens)

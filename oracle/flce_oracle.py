@@ -173,18 +173,23 @@ def forward(hidden, weight, labels, *, ignore_index: int = -100,
 
 def token_scales(valid: np.ndarray, reduction: str, num_label_tokens: int | None,
                  grad_loss) -> np.ndarray:
-    """d(loss)/d(token loss n): the upstream gradient through the reduction, 0 if ignored."""
-    valid_f = valid.astype(np.float64)
+    """d(loss)/d(token loss n): the upstream gradient through the reduction.
+
+    Exactly 0 at ignored positions, which contribute zero loss and zero
+    gradient (chunked_ce page, _ChunkedCrossEntropySum.forward, ``labels``);
+    with ``mean`` and no valid label there is nothing to scale, so all are 0.
+    """
     if reduction == "none":
-        return np.asarray(grad_loss, dtype=np.float64).reshape(-1) * valid_f
+        g = np.asarray(grad_loss, dtype=np.float64).reshape(-1)
+        return np.where(valid, g, 0.0)
     g = float(np.asarray(grad_loss, dtype=np.float64).reshape(-1)[0])
     if reduction == "sum":
         if num_label_tokens is not None:
             g /= float(num_label_tokens)
-        return g * valid_f
+        return np.where(valid, g, 0.0)
     if reduction == "mean":
         count = int(valid.sum())
-        return (g / count if count else float("nan")) * valid_f
+        return np.where(valid, g / count if count else 0.0, 0.0)
     raise ValueError(f"unknown reduction {reduction!r}")
 
 

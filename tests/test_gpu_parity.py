@@ -1,0 +1,222 @@
+"""GPU parity of the CUDA path (through the C ABI) against the FP64 oracle at
+sizes the oracle finishes in seconds: several tiles in every dimension, ragged
+tails, multiple backward vocabulary chunks, every reduction and the edge cases."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_projection_flce_b200 import flce
+from lm_head_projection_flce_b200 import workloads as W
+from oracle import flce_oracle as O
+
+from gpu_common import (GRAD_REL, LSE_ABS, assert_parity, gpu_device, max_rel, run_gpu,
+                        run_oracle, to_oracle)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return gpu_device()
+
+
+# ----------------------------------------------------------- GEMM self-test
+
+@pytest.mark.parametrize("a_mn", [False, True])
+@pytest.mark.parametrize("b_mn", [False, True])
+@pytest.mark.parametrize("mnk", [(128, 256, 64), (296, 264, 328), (1000, 1024, 520), (8, 8, 8)])
+def test_tensor_core_gemm_selftest(dev, a_mn, b_mn, mnk):
+    m, n, k = mnk
+    g = torch.Generator().manual_seed(m * 7 + n * 3 + k)
+    a = torch.randn(m, k, generator=g).to(torch.bfloat16)
+    b = torch.randn(n, k, generator=g).to(torch.bfloat16)
+    ref = a.float() @ b.float().T
+    a_dev = (a.T.contiguous() if a_mn else a).to(dev)
+    b_dev = (b.T.contiguous() if b_mn else b).to(dev)
+    d = flce.selftest_gemm(a_dev, b_dev, m, n, k, a_mn, b_mn)
+    torch.cuda.synchronize(dev)
+    assert torch.allclose(d.cpu(), ref, rtol=1e-4, atol=1e-3), float((d.cpu() - ref).abs().max())
+
+
+# ----------------------------------------------------------- parity cases
+
+CASES = {
+    "tiny": W.TINY,
+    "ragged_softcap_f32head": W.custom(333, 328, 1000, 1024, w_dtype="f32", softcap=30.0,
+                                       ignore_frac=0.1, seed=11),
+    "multi_tile": W.custom(1100, 1024, 8269, 8269, ignore_frac=0.05, seed=12),
+    "ktail_softcap_padded": W.custom(700, 520, 5000, 5120, softcap=30.0, ignore_frac=0.1,
+                                     w_sigma=0.05, seed=13),
+    "zipf_labels": W.custom(512, 256, 3000, 3000, label_dist="zipf", ignore_frac=0.2, seed=14),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity(dev, name):
+    w = CASES[name]
+    d = W.generate(w)
+    assert_parity(run_gpu(d, w, dev), run_oracle(d, w))
+
+
+@pytest.mark.parametrize("reduction,nlt", [("mean", None), ("none", None), ("sum", 977)])
+def test_reductions(dev, reduction, nlt):
+    w = CASES["ktail_softcap_padded"]
+    d = W.generate(w)
+    grad = None
+    if reduction == "none":
+        grad = torch.linspace(-1.0, 2.0, w.n_tokens, dtype=torch.float32)
+    else:
+        grad = torch.tensor([0.75])
+    got = run_gpu(d, w, dev, reduction=reduction, grad=grad, num_label_tokens=nlt)
+    ref = run_oracle(d, w, reduction=reduction, grad=grad, num_label_tokens=nlt)
+    assert_parity(got, ref)
+
+
+def test_multi_chunk_backward(dev):
+    """A smaller workspace makes the backward stream the vocabulary in narrower
+    chunks (down to 256 columns): same result within tolerance."""
+    w = CASES["multi_tile"]
+    d = W.generate(w)
+    ref = run_oracle(d, w)
+    lo = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, minimum=True)
+    hi = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab)
+    for ws in (lo, lo + 2 * w.n_tokens * 256 * 3, hi):
+        assert_parity(run_gpu(d, w, dev, ws_bytes=ws), ref)
+
+
+def test_outputs_stay_in_bounds(dev):
+    """Sentinels after every output and the workspace survive a ragged case."""
+    w = CASES["ragged_softcap_f32head"]
+    d = W.generate(w)
+    n, h, vp = w.n_tokens, w.hidden, w.padded_vocab
+    pad = 4096
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    sent = -12345.0
+    loss_b = torch.full((1 + pad,), sent, device=dev)
+    lse_b = torch.full((n + pad,), sent, device=dev)
+    dh_b = torch.full((n * h + pad,), sent, device=dev, dtype=torch.bfloat16)
+    dw_b = torch.full((vp * h + pad,), sent, device=dev, dtype=torch.float32)
+    ws_n = flce.workspace_size(n, h, vp, w.vocab, torch.float32)
+    ws_b = torch.full((ws_n + pad,), 0xA5, device=dev, dtype=torch.uint8)
+    loss, lse = flce.forward(hid, wt, lab, softcap=w.softcap, unpadded_vocab=w.vocab,
+                             workspace=ws_b[:ws_n], loss=loss_b[:1], lse=lse_b[:n])
+    dh, dw = flce.backward(hid, wt, lab, lse, torch.ones(1, device=dev), softcap=w.softcap,
+                           unpadded_vocab=w.vocab, workspace=ws_b[:ws_n],
+                           dhidden=dh_b[:n * h].view(n, h), dweight=dw_b[:vp * h].view(vp, h))
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
+    assert torch.all(loss_b[1:] == sent) and torch.all(lse_b[n:] == sent)
+    assert torch.all(dh_b[n * h:] == sent) and torch.all(dw_b[vp * h:] == sent)
+    assert torch.all(ws_b[ws_n:] == 0xA5)
+    ref = run_oracle(d, w)
+    assert float(np.max(np.abs(lse.double().cpu().numpy() - ref["lse"]))) <= LSE_ABS
+    assert max_rel(dh.double().cpu().numpy(), ref["dh"]) <= GRAD_REL
+    assert max_rel(dw.double().cpu().numpy(), ref["dw"]) <= GRAD_REL
+
+
+# ----------------------------------------------------------- edge cases
+
+def test_zero_tokens(dev):
+    w = W.custom(0, 64, 300, 320, seed=20)
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    loss, lse = flce.forward(hid, wt, lab, unpadded_vocab=w.vocab, reduction="sum")
+    mean, _ = flce.forward(hid, wt, lab, unpadded_vocab=w.vocab, reduction="mean")
+    none, _ = flce.forward(hid, wt, lab, unpadded_vocab=w.vocab, reduction="none")
+    dw = torch.full_like(wt, 7.0)
+    dh, dw = flce.backward(hid, wt, lab, lse, torch.ones(1, device=dev), unpadded_vocab=w.vocab,
+                           dweight=dw)
+    torch.cuda.synchronize(dev)
+    assert float(loss) == 0.0 and math.isnan(float(mean)) and none.numel() == 0
+    assert dh.numel() == 0 and torch.all(dw == 0)
+
+
+def test_all_tokens_ignored(dev):
+    w = W.custom(200, 128, 700, 768, ignore_frac=1.0, softcap=5.0, seed=21)
+    d = W.generate(w)
+    got = run_gpu(d, w, dev)
+    ref = run_oracle(d, w)
+    assert float(got["loss"].reshape(-1)[0]) == 0.0
+    assert np.all(got["dh"] == 0) and np.all(got["dw"] == 0)
+    assert float(np.max(np.abs(got["lse"] - ref["lse"]))) <= LSE_ABS
+    mean = run_gpu(d, w, dev, reduction="mean")
+    assert math.isnan(float(mean["loss"].reshape(-1)[0]))
+    assert np.all(mean["dh"] == 0) and np.all(mean["dw"] == 0)
+
+
+@pytest.mark.parametrize("softcap", [0.0, 3.0])
+def test_single_vocabulary_row(dev, softcap):
+    w = W.custom(150, 64, 1, 16, softcap=softcap, ignore_frac=0.2, seed=22)
+    d = W.generate(w)
+    got = run_gpu(d, w, dev)
+    ref = run_oracle(d, w)
+    assert float(np.max(np.abs(got["lse"] - ref["lse"]))) <= LSE_ABS
+    assert abs(float(got["loss"].reshape(-1)[0])) <= 1e-3
+    assert np.all(got["dw"][1:] == 0) and np.max(np.abs(got["dh"])) <= 1e-6
+
+
+def test_bad_labels_are_flagged_and_ignored(dev):
+    w = W.custom(300, 128, 900, 1024, softcap=0.0, seed=23)
+    d = W.generate(w)
+    bad = d["labels"].clone()
+    bad[3] = w.vocab + 5          # a padded row: never a valid target
+    bad[7] = -7
+    bad[100] = 10 ** 9
+    d_bad = dict(d, labels=bad)
+    got = run_gpu(d_bad, w, dev)
+    assert got["status"] == flce.FLCE_ERR_BAD_LABEL
+    assert flce.get_error(dev) == flce.FLCE_OK   # the word was cleared
+    fixed = bad.clone()
+    fixed[[3, 7, 100]] = W.IGNORE_INDEX
+    ref = run_oracle(dict(d, labels=fixed), w)
+    got["status"] = flce.FLCE_OK
+    assert_parity(got, ref)
+
+
+def test_pipeline_wait_timeout_is_reported(dev):
+    flce.selftest_wait_timeout(20000, dev)          # 20 ms wait that nothing satisfies
+    assert flce.get_error(dev) == flce.FLCE_ERR_TIMEOUT
+    # the context stays usable
+    w = W.TINY
+    d = W.generate(w)
+    assert_parity(run_gpu(d, w, dev), run_oracle(d, w))
+
+
+def test_no_nv_sized_allocation(dev):
+    """The call's own allocations (the workspace) stay far below N*V bytes."""
+    n, h, v = 4096, 1024, 128256
+    g = torch.Generator(device="cpu").manual_seed(5)
+    hid = torch.randn(n, h, generator=g).to(torch.bfloat16).to(dev)
+    wt = (torch.randn(v, h, generator=g) * 0.02).to(torch.bfloat16).to(dev)
+    lab = torch.randint(0, v, (n,), generator=g).to(dev)
+    loss = torch.empty(1, device=dev)
+    lse = torch.empty(n, device=dev)
+    dh = torch.empty_like(hid)
+    dw = torch.empty_like(wt)
+    grad = torch.ones(1, device=dev)
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    flce.forward(hid, wt, lab, loss=loss, lse=lse)
+    flce.backward(hid, wt, lab, lse, grad, dhidden=dh, dweight=dw)
+    torch.cuda.synchronize(dev)
+    extra = torch.cuda.max_memory_allocated(dev) - base
+    assert extra < n * v, (extra, n * v)
+    assert flce.get_error(dev) == flce.FLCE_OK
+
+
+def test_autograd_wrapper(dev):
+    w = CASES["ktail_softcap_padded"]
+    d = W.generate(w)
+    hid = d["hidden"].to(dev).requires_grad_(True)
+    wt = d["weight"].to(dev).requires_grad_(True)
+    lab = d["labels"].to(dev)
+    loss = flce.fused_linear_cross_entropy(hid, wt, lab, softcap=w.softcap, unpadded_vocab=w.vocab)
+    (2.0 * loss).backward()
+    torch.cuda.synchronize(dev)
+    ref = run_oracle(d, w, grad=torch.tensor([2.0]))
+    assert abs(float(loss) - float(ref["loss"])) <= 1e-4 * abs(float(ref["loss"]))
+    assert max_rel(hid.grad.double().cpu().numpy(), ref["dh"]) <= GRAD_REL
+    assert max_rel(wt.grad.double().cpu().numpy(), ref["dw"]) <= GRAD_REL
