@@ -157,6 +157,32 @@ int flce_selftest_gemm(const void* a, const void* b, float* d, int64_t m, int64_
  */
 int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream);
 
+/*
+ * Launch accounting for benchmarks (no counterpart on the pages).
+ *
+ * flce_launch_count: kernels this library has launched in this process.
+ * flce_profile_start: from now on, bracket every kernel launch of this library
+ *   with CUDA events on its stream (process-wide, any stream).  Returns
+ *   FLCE_ERR_INVALID_ARG if profiling is already on.
+ * flce_profile_stop: synchronise those events, stop recording and report one
+ *   flce_kernel_stat per kernel family that launched: launches, summed device
+ *   time between its events, and the algorithmic work the launches did
+ *   (FLOPs of the contraction; HBM bytes a single-pass kernel must move).
+ *   Writes at most `capacity` entries to `stats` and the family count to
+ *   *count.
+ */
+typedef struct {
+  char name[32];
+  int64_t launches;
+  double total_ms;
+  double flops;
+  double bytes;
+} flce_kernel_stat;
+
+unsigned long long flce_launch_count(void);
+int flce_profile_start(void);
+int flce_profile_stop(flce_kernel_stat* stats, int capacity, int* count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "flce.h"
 #include "epilogues.cuh"
@@ -279,6 +281,72 @@ static int device_info(DeviceInfo** out) {
   return FLCE_OK;
 }
 
+// ------------------------------------------------------------------ launch accounting
+// Every kernel launch is counted; while profiling is on, each launch is also
+// bracketed by CUDA events on its stream so a benchmark can report per-kernel
+// device time and algorithmic work without a profiler attached.
+
+enum KernelFamily {
+  KF_CAST = 0, KF_ZERO, KF_GEMM_FWD, KF_MERGE, KF_FINAL, KF_BWD_PREP, KF_GEMM_GRAD, KF_GEMM_DW,
+  KF_GEMM_DH, KF_SELFTEST_GEMM, KF_SELFTEST_WAIT, KF_COUNT
+};
+static const char* const kFamilyNames[KF_COUNT] = {
+    "cast_f32_bf16", "zero_rows",     "gemm_fwd_lse", "lse_merge",
+    "loss_finalize", "bwd_prep",      "gemm_bwd_grad", "gemm_bwd_dw",
+    "gemm_bwd_dh",   "selftest_gemm", "selftest_wait"};
+
+struct ProfRecord {
+  int family;
+  int device;
+  cudaEvent_t start, stop;
+  double flops, bytes;
+};
+
+static std::atomic<unsigned long long> g_launches{0};
+static std::mutex g_prof_mutex;
+static bool g_prof_on = false;
+static std::vector<ProfRecord> g_prof_records;
+static std::vector<cudaEvent_t> g_event_pool[64];
+
+static cudaEvent_t take_event(int dev) {
+  if (!g_event_pool[dev].empty()) {
+    cudaEvent_t e = g_event_pool[dev].back();
+    g_event_pool[dev].pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+class LaunchScope {
+ public:
+  LaunchScope(int family, double flops, double bytes, cudaStream_t st) : st_(st) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    if (!g_prof_on) return;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+    rec_.family = family;
+    rec_.device = dev;
+    rec_.flops = flops;
+    rec_.bytes = bytes;
+    rec_.start = take_event(dev);
+    rec_.stop = take_event(dev);
+    if (rec_.start && rec_.stop && cudaEventRecord(rec_.start, st_) == cudaSuccess) active_ = true;
+  }
+  ~LaunchScope() {
+    if (!active_) return;
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    if (cudaEventRecord(rec_.stop, st_) == cudaSuccess) g_prof_records.push_back(rec_);
+  }
+
+ private:
+  cudaStream_t st_;
+  ProfRecord rec_{};
+  bool active_ = false;
+};
+
 // 2-D BF16 tensor map, 128-byte swizzle, zero fill outside [inner, outer).
 static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
@@ -321,7 +389,8 @@ static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
 
 template <class Epi, bool kAMn, bool kBMn>
 static int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmShape g,
-                       const typename Epi::Params& ep, const DeviceInfo& dev, cudaStream_t st) {
+                       const typename Epi::Params& ep, const DeviceInfo& dev, cudaStream_t st,
+                       int family, double flops, double bytes) {
   g.raster = make_raster(g.m, g.n, g.k);
   g.tiles = int64_t(g.raster.m_tiles) * g.raster.n_tiles;
   g.err = dev.err;
@@ -332,6 +401,7 @@ static int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmShape g
                            int(kGemmSmemBytes)) != cudaSuccess)
     return FLCE_ERR_CUDA;
   const int grid = int(std::min<int64_t>(dev.num_sms, g.tiles));
+  LaunchScope scope(family, flops, bytes, st);
   kern<<<grid, kThreads, kGemmSmemBytes, st>>>(ta, tb, g, ep);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
@@ -340,6 +410,7 @@ static int launch_zero(void* p, size_t bytes, const DeviceInfo& dev, cudaStream_
   if (bytes == 0) return FLCE_OK;
   const int64_t n16 = int64_t(bytes / 16);
   const int grid = int(std::min<int64_t>(int64_t(dev.num_sms) * 8, cdiv(n16, 256)));
+  LaunchScope scope(KF_ZERO, 0.0, double(bytes), st);
   zero16_kernel<<<std::max(grid, 1), 256, 0, st>>>(static_cast<uint4*>(p), n16);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
@@ -349,6 +420,7 @@ static int launch_cast(const float* src, __nv_bfloat16* dst, int64_t elems,
   const int64_t n8 = elems / 8;
   if (n8 == 0) return FLCE_OK;
   const int grid = int(std::min<int64_t>(int64_t(dev.num_sms) * 8, cdiv(n8, 256)));
+  LaunchScope scope(KF_CAST, 0.0, double(elems) * 6.0, st);
   cast_f32_to_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
                                                 reinterpret_cast<uint4*>(dst), n8);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
@@ -498,6 +570,7 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
 
   if (n == 0) {
     if (reduction == FLCE_NONE) return FLCE_OK;
+    LaunchScope scope(KF_FINAL, 0.0, 4.0, cs);
     loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(blk_loss, blk_cnt, 0, reduction,
                                                       num_label_tokens, loss);
     return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
@@ -528,13 +601,20 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   ep.part_m = reinterpret_cast<float*>(ws + p.off_pm);
   ep.part_s = reinterpret_cast<float*>(ws + p.off_ps);
   ep.label_logit = reinterpret_cast<float*>(ws + p.off_zl);
-  if ((st = launch_gemm<EpiForward, false, false>(ta, tb, g, ep, *dev, cs)) != FLCE_OK) return st;
-
-  lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
-      ep.part_m, ep.part_s, int(p.v_tiles), n, ep.label_logit, labels, v, ignore_index, lse,
-      reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
+  const double fwd_flops = 2.0 * double(n) * double(v) * double(h);
+  const double fwd_bytes = 2.0 * (double(n) + double(v)) * double(h) + 8.0 * double(p.v_tiles) * n;
+  if ((st = launch_gemm<EpiForward, false, false>(ta, tb, g, ep, *dev, cs, KF_GEMM_FWD, fwd_flops,
+                                                  fwd_bytes)) != FLCE_OK)
+    return st;
+  {
+    LaunchScope scope(KF_MERGE, 0.0, 8.0 * double(p.v_tiles) * n + 24.0 * n, cs);
+    lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
+        ep.part_m, ep.part_s, int(p.v_tiles), n, ep.label_logit, labels, v, ignore_index, lse,
+        reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
+  }
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   if (reduction != FLCE_NONE) {
+    LaunchScope scope(KF_FINAL, 0.0, 12.0 * double(p.nblk), cs);
     loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(blk_loss, blk_cnt, int(p.nblk), reduction,
                                                       num_label_tokens, loss);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
@@ -595,8 +675,11 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
   float* scale = reinterpret_cast<float*>(ws + p.off_scale);
   float* dh32 = reinterpret_cast<float*>(ws + p.off_dh32);
   __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ws + p.off_g);
-  bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, n, v, ignore_index, reduction, num_label_tokens,
-                                      grad_loss, lse, lse2, scale, dev->err);
+  {
+    LaunchScope prep_scope(KF_BWD_PREP, 0.0, 24.0 * double(n), cs);
+    bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, n, v, ignore_index, reduction, num_label_tokens,
+                                        grad_loss, lse, lse2, scale, dev->err);
+  }
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
   CUtensorMap t_hid_k, t_w_k, t_hid_mn, t_w_mn;
@@ -628,7 +711,10 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
       ep.scale = scale;
       ep.g = gbuf;
       ep.ldg = vc;
-      if ((st = launch_gemm<EpiGrad, false, false>(t_hid_k, t_w_k, g, ep, *dev, cs)) != FLCE_OK)
+      const double fl = 2.0 * double(n) * double(width) * double(h);
+      const double by = 2.0 * (double(n) + double(width)) * double(h) + 2.0 * double(n) * gcols;
+      if ((st = launch_gemm<EpiGrad, false, false>(t_hid_k, t_w_k, g, ep, *dev, cs, KF_GEMM_GRAD,
+                                                   fl, by)) != FLCE_OK)
         return st;
     }
     CUtensorMap t_g_mn, t_g_k;
@@ -646,8 +732,10 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
       ep.rows = width;
       ep.cols = h;
       ep.f32 = w_dtype == FLCE_F32;
-      if ((st = launch_gemm<EpiStoreRows, true, true>(t_g_mn, t_hid_mn, g, ep, *dev, cs)) !=
-          FLCE_OK)
+      const double fl = 2.0 * double(n) * double(width) * double(h);
+      const double by = 2.0 * double(n) * (double(gcols) + double(h)) + double(wsz) * width * h;
+      if ((st = launch_gemm<EpiStoreRows, true, true>(t_g_mn, t_hid_mn, g, ep, *dev, cs,
+                                                      KF_GEMM_DW, fl, by)) != FLCE_OK)
         return st;
     }
     // K5: dhidden (+)= G . W[v0 : v0 + width]  (contraction over the chunk).
@@ -664,8 +752,11 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
       ep.rows = n;
       ep.cols = h;
       ep.mode = chunks == 1 ? 3 : (c == 0 ? 0 : (c == chunks - 1 ? 2 : 1));
-      if ((st = launch_gemm<EpiAccumRows, false, true>(t_g_k, t_w_mn, g, ep, *dev, cs)) !=
-          FLCE_OK)
+      const double fl = 2.0 * double(n) * double(width) * double(h);
+      const double rmw = ep.mode == 0 ? 4.0 : (ep.mode == 1 ? 8.0 : (ep.mode == 2 ? 6.0 : 2.0));
+      const double by = 2.0 * double(n) * gcols + 2.0 * double(width) * h + rmw * double(n) * h;
+      if ((st = launch_gemm<EpiAccumRows, false, true>(t_g_k, t_w_mn, g, ep, *dev, cs,
+                                                       KF_GEMM_DH, fl, by)) != FLCE_OK)
         return st;
     }
   }
@@ -714,10 +805,16 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   ep.rows = m;
   ep.cols = n;
   ep.f32 = 1;
-  if (!a_mn && !b_mn) return launch_gemm<EpiStoreRows, false, false>(ta, tb, g, ep, *dev, cs);
-  if (!a_mn && b_mn) return launch_gemm<EpiStoreRows, false, true>(ta, tb, g, ep, *dev, cs);
-  if (a_mn && !b_mn) return launch_gemm<EpiStoreRows, true, false>(ta, tb, g, ep, *dev, cs);
-  return launch_gemm<EpiStoreRows, true, true>(ta, tb, g, ep, *dev, cs);
+  const double fl = 2.0 * double(m) * double(n) * double(k);
+  const double by = 2.0 * (double(m) + double(n)) * double(k) + 4.0 * double(m) * n;
+  const int f = KF_SELFTEST_GEMM;
+  if (!a_mn && !b_mn)
+    return launch_gemm<EpiStoreRows, false, false>(ta, tb, g, ep, *dev, cs, f, fl, by);
+  if (!a_mn && b_mn)
+    return launch_gemm<EpiStoreRows, false, true>(ta, tb, g, ep, *dev, cs, f, fl, by);
+  if (a_mn && !b_mn)
+    return launch_gemm<EpiStoreRows, true, false>(ta, tb, g, ep, *dev, cs, f, fl, by);
+  return launch_gemm<EpiStoreRows, true, true>(ta, tb, g, ep, *dev, cs, f, fl, by);
 }
 
 extern "C" int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream) {
@@ -725,7 +822,64 @@ extern "C" int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t
   DeviceInfo* dev = nullptr;
   int st = device_info(&dev);
   if (st != FLCE_OK) return st;
+  LaunchScope scope(KF_SELFTEST_WAIT, 0.0, 0.0, static_cast<cudaStream_t>(stream));
   wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       dev->err, uint64_t(timeout_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+extern "C" unsigned long long flce_launch_count(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
+
+extern "C" int flce_profile_start(void) {
+  std::lock_guard<std::mutex> lock(g_prof_mutex);
+  if (g_prof_on) return FLCE_ERR_INVALID_ARG;
+  g_prof_on = true;
+  return FLCE_OK;
+}
+
+extern "C" int flce_profile_stop(flce_kernel_stat* stats, int capacity, int* count) {
+  std::vector<ProfRecord> recs;
+  {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    if (!g_prof_on) return FLCE_ERR_INVALID_ARG;
+    g_prof_on = false;
+    recs.swap(g_prof_records);
+  }
+  double ms[KF_COUNT] = {0}, fl[KF_COUNT] = {0}, by[KF_COUNT] = {0};
+  int64_t nl[KF_COUNT] = {0};
+  int status = FLCE_OK;
+  for (const ProfRecord& r : recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+      status = FLCE_ERR_CUDA;
+    ms[r.family] += t;
+    fl[r.family] += r.flops;
+    by[r.family] += r.bytes;
+    nl[r.family] += 1;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    for (const ProfRecord& r : recs) {
+      g_event_pool[r.device].push_back(r.start);
+      g_event_pool[r.device].push_back(r.stop);
+    }
+  }
+  int k = 0;
+  for (int f = 0; f < KF_COUNT; ++f) {
+    if (nl[f] == 0) continue;
+    if (stats != nullptr && k < capacity) {
+      std::memset(&stats[k], 0, sizeof(flce_kernel_stat));
+      std::strncpy(stats[k].name, kFamilyNames[f], sizeof(stats[k].name) - 1);
+      stats[k].launches = nl[f];
+      stats[k].total_ms = ms[f];
+      stats[k].flops = fl[f];
+      stats[k].bytes = by[f];
+    }
+    ++k;
+  }
+  if (count) *count = k;
+  return status;
 }

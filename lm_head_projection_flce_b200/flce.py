@@ -56,7 +56,16 @@ SIGNATURES = {
     "flce_selftest_gemm": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_int,
                                     _c_int, _c_ptr]),
     "flce_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _c_ptr]),
+    "flce_launch_count": (ctypes.c_ulonglong, []),
+    "flce_profile_start": (_c_int, []),
+    "flce_profile_stop": (_c_int, [_c_ptr, _c_int, ctypes.POINTER(_c_int)]),
 }
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
 
 _LIB = None
 
@@ -238,3 +247,29 @@ def fused_linear_cross_entropy(hidden, weight, labels, *, ignore_index: int = -1
     """Autograd-aware loss: gradients flow to ``hidden`` and ``weight``."""
     return _FusedLinearCE.apply(hidden, weight, labels, ignore_index, softcap, unpadded_vocab,
                                 reduction, num_label_tokens)
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(load_library().flce_launch_count())
+
+
+def profile_start() -> None:
+    """Bracket every library kernel launch with CUDA events until profile_stop()."""
+    _check("flce_profile_start", load_library().flce_profile_start())
+
+
+def profile_stop() -> dict:
+    """Per kernel family: launches, device ms (CUDA events) and algorithmic work."""
+    lib = load_library()
+    cap = 32
+    arr = (KernelStat * cap)()
+    count = _c_int(0)
+    _check("flce_profile_stop", lib.flce_profile_stop(ctypes.cast(arr, _c_ptr), cap,
+                                                       ctypes.byref(count)))
+    out = {}
+    for i in range(min(count.value, cap)):
+        st = arr[i]
+        out[st.name.decode()] = {"launches": int(st.launches), "total_ms": float(st.total_ms),
+                                 "flops": float(st.flops), "bytes": float(st.bytes)}
+    return out

@@ -97,6 +97,13 @@ LARGE_HEAD = _register(Workload(
 # Ordered as listed above.
 WORKLOAD_ORDER = [TINY, LLAMA_HEAD, SOFTCAP_F32_HEAD, LONG_SEQ, LARGE_HEAD]
 
+# A reduced case for profiler captures: the head (268 MB) is still larger than
+# L2, so DRAM counters mean something, but the whole run holds under 1 GB.
+PROFILE_CASE = _register(Workload(
+    name="profile_n2048_h4096_v32768", n_tokens=2048, hidden=4096, vocab=32768,
+    padded_vocab=32768, batch=1, seq=2048, w_sigma=0.02, ignore_frac=0.05, softcap=0.0,
+    reduction="sum", normalize_by_label_tokens=True, seed=2001))
+
 
 def custom(n_tokens: int, hidden: int, vocab: int, padded_vocab: int | None = None,
            **kw) -> Workload:
