@@ -227,15 +227,17 @@ def cpu_baseline(w, d, target_s: float = 15.0, max_tokens: int = 512) -> dict:
     hidden, weight, labels = oracle_inputs(d)
     nlt = d["num_label_tokens"] if w.normalize_by_label_tokens else None
     rng = np.random.default_rng(7)
-    probe = rng.choice(w.n_tokens, size=min(8, w.n_tokens), replace=False)
-    t0 = time.perf_counter()
-    oracle_step(O, w, hidden, weight, labels, probe, nlt)
-    t_probe = time.perf_counter() - t0
-    s = int(min(max_tokens, w.n_tokens, max(8, target_s / max(t_probe, 1e-3) * len(probe))))
-    rows = rng.choice(w.n_tokens, size=s, replace=False)
-    t0 = time.perf_counter()
-    oracle_step(O, w, hidden, weight, labels, rows, nlt)
-    dt = time.perf_counter() - t0
+    # Grow the sample (x4) until one oracle pass takes about target_s / 4 or more;
+    # the oracle has a fixed per-call cost (the full [Vp, H] dW), so probe sizes grow.
+    s = min(16, w.n_tokens)
+    while True:
+        rows = rng.choice(w.n_tokens, size=s, replace=False)
+        t0 = time.perf_counter()
+        oracle_step(O, w, hidden, weight, labels, rows, nlt)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or s >= min(max_tokens, w.n_tokens):
+            break
+        s = min(4 * s, max_tokens, w.n_tokens)
     return {"value": s / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": (f"{s} seeded tokens of {w.name} through the FP64 oracle's full forward + "
                        f"backward (lse over all {w.vocab} rows, their dhidden rows and their "
