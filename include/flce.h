@@ -158,6 +158,34 @@ int flce_selftest_gemm(const void* a, const void* b, float* d, int64_t m, int64_
 int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream);
 
 /*
+ * Forward that allocates nothing and takes no workspace (the pages have no
+ * counterpart; it exists for callers that cannot supply scratch memory, such
+ * as a plugin inside a framework whose allocator owns the whole device, or a
+ * service that allows no device allocation once running).
+ *   Arguments and results are those of flce_forward without workspace /
+ *   ws_bytes; the caller still passes every input and output.
+ *   Scratch: a 32 MiB array in this library's device memory, present on every
+ *   GPU that loads the library until the process exits.  A problem whose
+ *   forward scratch (8 B x ceil(V/256) x N for the logsumexp partials, plus
+ *   4 B x N, plus the BF16 copy of an FP32 head) exceeds 32 MiB is refused
+ *   with FLCE_ERR_WORKSPACE and nothing is enqueued; e.g. N = 4096 tokens with
+ *   V = 128256 and a BF16 head needs 16.5 MiB and fits.
+ *   The array is shared by every call on a device and keeps whatever the last
+ *   call left in it; the forward writes every scratch byte before reading it,
+ *   so nothing has to be cleared between calls.  Calls that overlap on the GPU
+ *   (different streams, or different host threads) race on the array: order
+ *   them on one stream or synchronise between them.
+ *   The first call on each device looks up the array's device address with
+ *   cudaGetSymbolAddress (with that device current); make that first call
+ *   before any stream capture.
+ */
+int flce_forward_noalloc(const void* hidden, const void* weight, int w_dtype,
+                         const int64_t* labels, int64_t n_tokens, int64_t hidden_size,
+                         int64_t padded_vocab, int64_t unpadded_vocab, int64_t ignore_index,
+                         float softcap, int reduction, int64_t num_label_tokens, float* loss,
+                         float* lse, flce_stream_t stream);
+
+/*
  * Launch accounting for benchmarks (no counterpart on the pages).
  *
  * flce_launch_count: kernels this library has launched in this process.

@@ -883,3 +883,56 @@ extern "C" int flce_profile_stop(flce_kernel_stat* stats, int capacity, int* cou
   if (count) *count = k;
   return status;
 }
+
+// ================================================== forward without allocation
+//
+// For callers that cannot hand this library any device memory of their own
+// beyond inputs and outputs: for example a plugin running inside another
+// framework whose allocator owns the whole device and offers no scratch API,
+// or a service that forbids device allocations after start-up because one
+// that fails mid-run cannot be recovered.  The forward's scratch (per-tile
+// logsumexp partials, the label logits and the loss block sums) then lives in
+// a fixed array in this library's own device memory instead of a workspace.
+
+namespace flce {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB on every device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static std::mutex g_noalloc_mutex;
+static void* g_noalloc_addr[64];  // device address of g_noalloc_scratch, per device
+
+}  // namespace flce
+
+extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int w_dtype,
+                                    const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                                    int64_t unpadded, int64_t ignore_index, float softcap,
+                                    int reduction, int64_t num_label_tokens, float* loss,
+                                    float* lse, flce_stream_t stream) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  if (!shape_ok(n, h, vp, v, w_dtype)) return FLCE_ERR_INVALID_ARG;
+  // The whole scratch must fit the fixed array; nothing here can grow it.
+  if (plan_forward(Shape{n, h, vp, v, w_dtype}).total > kNoAllocScratchBytes)
+    return FLCE_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FLCE_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    // First call on a device: look up where the array lives on it.  In host
+    // code the array's name is only a host-side stand-in, never a device
+    // address, so the kernels get this looked-up pointer instead.
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return FLCE_ERR_CUDA;
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  // Same kernels, same results as flce_forward; every scratch byte the
+  // forward reads is written earlier in the same call, so the array's stale
+  // contents from a previous call never need clearing.
+  return flce_forward(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index, softcap,
+                      reduction, num_label_tokens, loss, lse, scratch, kNoAllocScratchBytes,
+                      stream);
+}

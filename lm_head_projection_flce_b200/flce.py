@@ -56,6 +56,9 @@ SIGNATURES = {
     "flce_selftest_gemm": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_int,
                                     _c_int, _c_ptr]),
     "flce_selftest_wait_timeout": (_c_int, [ctypes.c_uint, _c_ptr]),
+    "flce_forward_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64,
+                                      _c_i64, _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr,
+                                      _c_ptr, _c_ptr]),
     "flce_launch_count": (ctypes.c_ulonglong, []),
     "flce_profile_start": (_c_int, []),
     "flce_profile_stop": (_c_int, [_c_ptr, _c_int, ctypes.POINTER(_c_int)]),
@@ -273,3 +276,28 @@ def profile_stop() -> dict:
         out[st.name.decode()] = {"launches": int(st.launches), "total_ms": float(st.total_ms),
                                  "flops": float(st.flops), "bytes": float(st.bytes)}
     return out
+
+
+def forward_noalloc(hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
+                    unpadded_vocab: int | None = None, reduction: str = "sum",
+                    num_label_tokens: int | None = None, loss: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, stream=None):
+    """flce_forward_noalloc: the forward with the library's fixed 32 MiB device
+    scratch instead of a workspace, for callers that cannot provide scratch
+    memory.  Only the outputs are allocated here (when not given)."""
+    lib = load_library()
+    hid, lab = _prepare(hidden, weight, labels)
+    n, h = hid.shape
+    vp = weight.shape[0]
+    v = _vocab(weight, unpadded_vocab)
+    dev = hid.device
+    if loss is None:
+        loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(n, dtype=torch.float32, device=dev)
+    st = lib.flce_forward_noalloc(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n,
+                                  h, vp, v, ignore_index, float(softcap), REDUCTIONS[reduction],
+                                  int(num_label_tokens or 0), _ptr(loss), _ptr(lse),
+                                  _stream_handle(dev, stream))
+    _check("flce_forward_noalloc", st)
+    return (loss if reduction == "none" else loss.reshape(())), lse
