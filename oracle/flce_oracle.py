@@ -63,13 +63,13 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     names for an FP32 head ("the cast FSDP applies", i.e. ``tensor.to(bfloat16)``).
     """
     f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    keep_lsb = (u >> np.uint64(16)) & np.uint64(1)
-    r = ((u + np.uint64(0x7FFF) + keep_lsb) >> np.uint64(16)) << np.uint64(16)
-    r = r.astype(np.uint32)
+    u = f.view(np.uint32)
+    # For every non-NaN encoding u <= 0xFF800000, so u + 0x7FFF + 1 stays below 2**32.
+    keep_lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = ((u + np.uint32(0x7FFF) + keep_lsb) >> np.uint32(16)) << np.uint32(16)
     nan = np.isnan(f)
     if nan.any():
-        r[nan] = (u[nan].astype(np.uint32) & np.uint32(0xFFFF0000)) | np.uint32(0x00400000)
+        r[nan] = (u[nan] & np.uint32(0xFFFF0000)) | np.uint32(0x00400000)
     return r.view(np.float32).astype(np.float64)
 
 
@@ -81,7 +81,10 @@ def compute_head(weight: np.ndarray, unpadded_vocab: int) -> np.ndarray:
     """
     rows = weight[:unpadded_vocab]
     if rows.dtype == np.float32:
-        return bf16_round(rows)
+        out = np.empty(rows.shape, dtype=np.float64)
+        for s in range(0, rows.shape[0], 8192):      # elementwise; blocks only bound memory
+            out[s:s + 8192] = bf16_round(rows[s:s + 8192])
+        return out
     return np.asarray(rows, dtype=np.float64)
 
 
