@@ -265,3 +265,33 @@ struct EpiAccumRows {
 };
 
 }  // namespace flce
+
+namespace flce {
+
+// The epilogues a grouped launch may run, selected per problem at run time.
+// kKinds is a bit mask of the EpiKind values compiled into the kernel.
+template <int kKinds>
+struct EpiSet {
+  EpiForward::Params fwd;
+  EpiGrad::Params grad;
+  EpiStoreRows::Params store;
+  EpiAccumRows::Params accum;
+
+  static __device__ __forceinline__ void dispatch(int kind, const EpiSet& e, uint32_t taddr,
+                                                  int mt, int nt, int row) {
+    if ((kKinds & (1 << kEpiForward)) && kind == kEpiForward)
+      EpiForward::tile(e.fwd, taddr, mt, nt, row);
+    else if ((kKinds & (1 << kEpiGrad)) && kind == kEpiGrad)
+      EpiGrad::tile(e.grad, taddr, mt, nt, row);
+    else if ((kKinds & (1 << kEpiStoreRows)) && kind == kEpiStoreRows)
+      EpiStoreRows::tile(e.store, taddr, mt, nt, row);
+    else if ((kKinds & (1 << kEpiAccumRows)) && kind == kEpiAccumRows)
+      EpiAccumRows::tile(e.accum, taddr, mt, nt, row);
+  }
+};
+
+constexpr int kEpiSetForward = 1 << kEpiForward;
+constexpr int kEpiSetBackward = (1 << kEpiGrad) | (1 << kEpiStoreRows) | (1 << kEpiAccumRows);
+constexpr int kEpiSetStore = 1 << kEpiStoreRows;
+
+}  // namespace flce

@@ -11,13 +11,16 @@
 //   K2b     deterministic final sum -> loss (/ num_label_tokens, or mean)
 // Backward (nemo_automodel.components.loss.chunked_ce,
 //           _ChunkedCrossEntropySum.backward: recompute instead of storing):
-//   prep    per-token gradient scale s_n, lse * log2(e)
-//   per vocabulary chunk [v0, v0 + Vc):
+//   prep    per-token gradient scale s_n, lse * log2(e), zero tile counters
+//   per vocabulary chunk c = [v0, v0 + Vc), G double-buffered (G[c % 2]):
 //     K3    GEMM hidden . W[chunk]^T, epilogue: G = s_n (softmax - onehot) dcap
 //           -> BF16 G[N, Vc] (bounded chunk buffer, never [N, V])
-//     K4    GEMM G^T . hidden  -> dW[chunk] (head dtype)
 //     K5    GEMM G . W[chunk]  -> dhidden, FP32 accumulation across chunks,
 //           BF16 on the last chunk
+//     K4    GEMM G^T . hidden  -> dW[chunk] (head dtype)
+//   launched as K3(0), then one grouped launch per chunk {K5(c), K4(c),
+//   K3(c+1)} whose CTAs take tiles dynamically, long K5 tiles first, so no
+//   launch ends on a partial wave of long tiles
 //   zero    dW rows [V, Vp)
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -46,7 +49,7 @@ constexpr int kMergeWarps = 8;
 constexpr int kFinalThreads = 256;
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1024;  // TMA coordinates are int32
 constexpr size_t kAlign = 1024;
-constexpr size_t kChunkBudgetBytes = size_t(256) << 20;  // default G chunk buffer
+constexpr size_t kChunkBudgetBytes = size_t(128) << 20;  // default size of each G buffer
 constexpr int64_t kMinChunk = 4096;
 
 // ------------------------------------------------------------------ kernels
@@ -176,8 +179,10 @@ __global__ void __launch_bounds__(1024)
                     int64_t ignore_index, int reduction, int64_t num_label_tokens,
                     const float* __restrict__ grad_loss, const float* __restrict__ lse,
                     float* __restrict__ lse2, float* __restrict__ scale,
+                    unsigned* __restrict__ counters, int n_counters,
                     unsigned* __restrict__ err) {
   __shared__ int warp_cnt[32];
+  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0u;
   int cnt = 0;
   bool bad = false;
   for (int64_t n = threadIdx.x; n < n_tokens; n += blockDim.x) {
@@ -223,10 +228,7 @@ __global__ void wait_timeout_selftest_kernel(unsigned* err, uint64_t timeout_ns)
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    GemmShape g{};
-    g.err = err;
-    g.timeout_ns = timeout_ns;
-    wait_phase(smem_u32(&bar), 0, &ctl, g);
+    wait_phase(smem_u32(&bar), 0, &ctl, err, timeout_ns);
   }
   __syncthreads();
 }
@@ -288,12 +290,12 @@ static int device_info(DeviceInfo** out) {
 
 enum KernelFamily {
   KF_CAST = 0, KF_ZERO, KF_GEMM_FWD, KF_MERGE, KF_FINAL, KF_BWD_PREP, KF_GEMM_GRAD, KF_GEMM_DW,
-  KF_GEMM_DH, KF_SELFTEST_GEMM, KF_SELFTEST_WAIT, KF_COUNT
+  KF_GEMM_DH, KF_SELFTEST_GEMM, KF_SELFTEST_WAIT, KF_GEMM_BWD, KF_COUNT
 };
 static const char* const kFamilyNames[KF_COUNT] = {
     "cast_f32_bf16", "zero_rows",     "gemm_fwd_lse", "lse_merge",
     "loss_finalize", "bwd_prep",      "gemm_bwd_grad", "gemm_bwd_dw",
-    "gemm_bwd_dh",   "selftest_gemm", "selftest_wait"};
+    "gemm_bwd_dh",   "selftest_gemm", "selftest_wait", "gemm_bwd_fused"};
 
 struct ProfRecord {
   int family;
@@ -376,33 +378,78 @@ static bool tmap_mnmajor(CUtensorMap* tm, const void* base, int64_t mn, int64_t 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Raster that keeps operand panels resident in L2: when all of B (or all of A)
+// fits in the budget, iterate over its tiles fastest so it is read from HBM
+// once while the other operand streams; otherwise group m-tiles whose A panels
+// fit.
+constexpr int64_t kL2ResidentBytes = int64_t(40) << 20;
+
 static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
-  TileRaster r;
+  TileRaster r{};
   r.m_tiles = int(cdiv(m, kBM));
   r.n_tiles = int(cdiv(n, kBN));
-  // Keep the group's A panel (group_m x 128 rows x K) around 48 MB so it stays in L2.
-  const int64_t panel = int64_t(kBM) * std::max<int64_t>(k, 1) * 2;
-  int64_t gm = std::max<int64_t>(1, (int64_t(48) << 20) / panel);
-  r.group_m = int(std::min<int64_t>(gm, r.m_tiles));
+  const int64_t kk = std::max<int64_t>(k, 1);
+  const int64_t a_panel = int64_t(kBM) * kk * 2, b_panel = int64_t(kBN) * kk * 2;
+  const int64_t a_all = a_panel * r.m_tiles, b_all = b_panel * r.n_tiles;
+  if (a_all <= kL2ResidentBytes && a_all <= b_all) {
+    r.n_fast = 0;
+    r.group = r.m_tiles;
+  } else if (b_all <= kL2ResidentBytes) {
+    r.n_fast = 1;
+    r.group = r.n_tiles;
+  } else {
+    r.n_fast = 0;
+    r.group = int(std::min<int64_t>(std::max<int64_t>(1, (int64_t(24) << 20) / a_panel), r.m_tiles));
+  }
   return r;
 }
 
-template <class Epi, bool kAMn, bool kBMn>
-static int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmShape g,
-                       const typename Epi::Params& ep, const DeviceInfo& dev, cudaStream_t st,
-                       int family, double flops, double bytes) {
-  g.raster = make_raster(g.m, g.n, g.k);
-  g.tiles = int64_t(g.raster.m_tiles) * g.raster.n_tiles;
+static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool b_mn, int epi) {
+  GemmProblem p{};
+  p.m = m;
+  p.n = n;
+  p.k = k;
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
+  p.epi = epi;
+  p.num_kb = int(cdiv(k, kBK));
+  p.raster = make_raster(m, n, k);
+  p.tiles = (m > 0 && n > 0) ? int64_t(p.raster.m_tiles) * p.raster.n_tiles : 0;
+  return p;
+}
+
+// One persistent launch over up to kMaxProblems problems; tiles taken from
+// `counter` (zeroed beforehand) when given, else round robin.
+// Problem i runs with configuration Ci (its slot is fixed even when it has no
+// tiles, so the compile-time configuration always matches).
+template <int kKinds, class C0, class C1 = NoProblem, class C2 = NoProblem>
+static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
+                        const CUtensorMap* maps_b, int count, const EpiSet<kKinds>& ep,
+                        unsigned* counter, const DeviceInfo& dev, cudaStream_t st, int family,
+                        double flops, double bytes) {
+  GemmMaps maps;
+  GemmGroup g{};
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    g.prob[i] = probs[i];
+    g.prob[i].tile_begin = total;
+    total += probs[i].tiles;
+    maps.a[i] = maps_a[i];
+    maps.b[i] = maps_b[i];
+  }
+  g.num_problems = count;
+  if (total == 0) return FLCE_OK;
+  g.total_tiles = total;
+  g.tile_counter = counter;
   g.err = dev.err;
   g.timeout_ns = kDefaultTimeoutNs;
-  if (g.tiles == 0) return FLCE_OK;
-  auto kern = tc_gemm_kernel<Epi, kAMn, kBMn>;
+  auto kern = tc_gemm_group_kernel<EpiSet<kKinds>, C0, C1, C2>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(kGemmSmemBytes)) != cudaSuccess)
     return FLCE_ERR_CUDA;
-  const int grid = int(std::min<int64_t>(dev.num_sms, g.tiles));
+  const int grid = int(std::min<int64_t>(dev.num_sms, total));
   LaunchScope scope(family, flops, bytes, st);
-  kern<<<grid, kThreads, kGemmSmemBytes, st>>>(ta, tb, g, ep);
+  kern<<<grid, kThreads, kGemmSmemBytes, st>>>(maps, g, ep);
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -440,7 +487,8 @@ struct FwdPlan {
 
 struct BwdPlan {
   int64_t vc;  // vocabulary chunk width (multiple of 256)
-  size_t off_lse2, off_scale, off_dh32, off_wb, off_g, fixed, total;
+  int64_t n_counters;
+  size_t off_lse2, off_scale, off_cnt, off_dh32, off_wb, off_g, fixed, total;
 };
 
 static FwdPlan plan_forward(const Shape& s) {
@@ -471,10 +519,12 @@ static BwdPlan plan_backward(const Shape& s, int64_t vc) {
   size_t o = 0;
   p.off_lse2 = o;  o = align_up(o + size_t(s.n) * 4);
   p.off_scale = o; o = align_up(o + size_t(s.n) * 4);
+  p.n_counters = cdiv(s.v, kBN) + 2;  // one per launch at the narrowest chunking
+  p.off_cnt = o;   o = align_up(o + size_t(p.n_counters) * 4);
   p.off_dh32 = o;  o = align_up(o + size_t(s.n) * s.h * 4);
   p.off_wb = o;    o = align_up(o + (s.w_dtype == FLCE_F32 ? size_t(s.v) * s.h * 2 : 0));
   p.fixed = o;
-  p.off_g = o;     o = align_up(o + size_t(s.n) * vc * 2);
+  p.off_g = o;     o = align_up(o + 2 * size_t(s.n) * vc * 2);  // two chunk buffers
   p.total = o;
   return p;
 }
@@ -588,11 +638,9 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   CUtensorMap ta, tb;
   if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBN))
     return FLCE_ERR_CUDA;
-  GemmShape g{};
-  g.m = n;
-  g.n = v;
-  g.k = h;
-  EpiForward::Params ep{};
+  const GemmProblem prob = make_problem(n, v, h, false, false, kEpiForward);
+  EpiSet<kEpiSetForward> es{};
+  EpiForward::Params& ep = es.fwd;
   ep.labels = labels;
   ep.n_tokens = n;
   ep.vocab = v;
@@ -603,8 +651,9 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   ep.label_logit = reinterpret_cast<float*>(ws + p.off_zl);
   const double fwd_flops = 2.0 * double(n) * double(v) * double(h);
   const double fwd_bytes = 2.0 * (double(n) + double(v)) * double(h) + 8.0 * double(p.v_tiles) * n;
-  if ((st = launch_gemm<EpiForward, false, false>(ta, tb, g, ep, *dev, cs, KF_GEMM_FWD, fwd_flops,
-                                                  fwd_bytes)) != FLCE_OK)
+  if ((st = launch_group<kEpiSetForward, ProblemCfg<false, false, kEpiForward>>(
+           &prob, &ta, &tb, 1, es, nullptr, *dev, cs, KF_GEMM_FWD, fwd_flops, fwd_bytes)) !=
+      FLCE_OK)
     return st;
   {
     LaunchScope scope(KF_MERGE, 0.0, 8.0 * double(p.v_tiles) * n + 24.0 * n, cs);
@@ -645,7 +694,8 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
   // Widest chunk that fits the workspace, up to the default.
   int64_t vc = default_chunk(s);
   if (n > 0) {
-    const int64_t fit = int64_t((ws_bytes - p0.fixed) / (2 * size_t(n))) / kBN * kBN;
+    // two chunk buffers of n x vc BF16
+    const int64_t fit = int64_t((ws_bytes - p0.fixed) / (4 * size_t(n))) / kBN * kBN;
     vc = std::max<int64_t>(kBN, std::min(vc, fit));
   }
   const BwdPlan p = plan_backward(s, vc);
@@ -674,11 +724,14 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
   float* lse2 = reinterpret_cast<float*>(ws + p.off_lse2);
   float* scale = reinterpret_cast<float*>(ws + p.off_scale);
   float* dh32 = reinterpret_cast<float*>(ws + p.off_dh32);
-  __nv_bfloat16* gbuf = reinterpret_cast<__nv_bfloat16*>(ws + p.off_g);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + p.off_cnt);
+  __nv_bfloat16* gbufs[2] = {reinterpret_cast<__nv_bfloat16*>(ws + p.off_g),
+                             reinterpret_cast<__nv_bfloat16*>(ws + p.off_g) + size_t(n) * vc};
   {
     LaunchScope prep_scope(KF_BWD_PREP, 0.0, 24.0 * double(n), cs);
     bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, n, v, ignore_index, reduction, num_label_tokens,
-                                        grad_loss, lse, lse2, scale, dev->err);
+                                        grad_loss, lse, lse2, scale, counters,
+                                        int(p.n_counters), dev->err);
   }
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
@@ -687,78 +740,100 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
       !tmap_mnmajor(&t_hid_mn, hidden, h, n, h) || !tmap_mnmajor(&t_w_mn, wb, h, v, h))
     return FLCE_ERR_CUDA;
 
+  using CfgGrad = ProblemCfg<false, false, kEpiGrad>;
+  using CfgDh = ProblemCfg<false, true, kEpiAccumRows>;
+  using CfgDw = ProblemCfg<true, true, kEpiStoreRows>;
   const int64_t chunks = cdiv(v, vc);
-  for (int64_t c = 0; c < chunks; ++c) {
-    const int64_t v0 = c * vc;
-    const int64_t width = std::min(vc, v - v0);
-    const int64_t gcols = cdiv(width, kBN) * kBN;
+  auto chunk_v0 = [&](int64_t c) { return c * vc; };
+  auto chunk_width = [&](int64_t c) { return std::min(vc, v - c * vc); };
+  auto chunk_gcols = [&](int64_t c) { return cdiv(chunk_width(c), kBN) * kBN; };
+  const float softcap_k = softcap > 0.0f ? 2.0f * kLog2e / softcap : 0.0f;
 
-    // K3: recompute logits for the chunk and form G (BF16) in the chunk buffer.
-    {
-      GemmShape g{};
-      g.m = n;
-      g.n = width;
-      g.k = h;
-      g.b_mn_off = int(v0);
-      EpiGrad::Params ep{};
-      ep.labels = labels;
-      ep.n_tokens = n;
-      ep.vocab = v;
-      ep.v0 = v0;
-      ep.softcap = softcap;
-      ep.softcap_k = softcap > 0.0f ? 2.0f * kLog2e / softcap : 0.0f;
-      ep.lse2 = lse2;
-      ep.scale = scale;
-      ep.g = gbuf;
-      ep.ldg = vc;
-      const double fl = 2.0 * double(n) * double(width) * double(h);
-      const double by = 2.0 * (double(n) + double(width)) * double(h) + 2.0 * double(n) * gcols;
-      if ((st = launch_gemm<EpiGrad, false, false>(t_hid_k, t_w_k, g, ep, *dev, cs, KF_GEMM_GRAD,
-                                                   fl, by)) != FLCE_OK)
-        return st;
-    }
+  // K3 for chunk c: problem, maps and epilogue parameters.
+  auto grad_problem = [&](int64_t c, GemmProblem* pr, CUtensorMap* ma, CUtensorMap* mb,
+                          EpiGrad::Params* ep) {
+    *pr = make_problem(n, chunk_width(c), h, false, false, kEpiGrad);
+    pr->b_mn_off = int(chunk_v0(c));
+    *ma = t_hid_k;
+    *mb = t_w_k;
+    ep->labels = labels;
+    ep->n_tokens = n;
+    ep->vocab = v;
+    ep->v0 = chunk_v0(c);
+    ep->softcap = softcap;
+    ep->softcap_k = softcap_k;
+    ep->lse2 = lse2;
+    ep->scale = scale;
+    ep->g = gbufs[c & 1];
+    ep->ldg = vc;
+  };
+  auto grad_flops = [&](int64_t c) { return 2.0 * double(n) * double(chunk_width(c)) * double(h); };
+  auto grad_bytes = [&](int64_t c) {
+    return 2.0 * (double(n) + double(chunk_width(c))) * double(h) +
+           2.0 * double(n) * double(chunk_gcols(c));
+  };
+
+  {  // K3 of the first chunk on its own
+    GemmProblem pr;
+    CUtensorMap ma, mb;
+    EpiSet<kEpiSetBackward> es{};
+    grad_problem(0, &pr, &ma, &mb, &es.grad);
+    if ((st = launch_group<kEpiSetBackward, CfgGrad>(&pr, &ma, &mb, 1, es, &counters[0], *dev, cs,
+                                                     KF_GEMM_GRAD, grad_flops(0),
+                                                     grad_bytes(0))) != FLCE_OK)
+      return st;
+  }
+  for (int64_t c = 0; c < chunks; ++c) {
+    const int64_t v0 = chunk_v0(c), width = chunk_width(c), gcols = chunk_gcols(c);
+    __nv_bfloat16* gbuf = gbufs[c & 1];
     CUtensorMap t_g_mn, t_g_k;
     if (!tmap_mnmajor(&t_g_mn, gbuf, gcols, n, vc) || !tmap_kmajor(&t_g_k, gbuf, gcols, n, vc, kBM))
       return FLCE_ERR_CUDA;
-    // K4: dW[v0 : v0 + width] = G^T . hidden  (contraction over tokens).
+    GemmProblem pr[3];
+    CUtensorMap ma[3], mb[3];
+    EpiSet<kEpiSetBackward> es{};
+    int count = 0;
+    double flops = 0.0, bytes = 0.0;
+    // K5: dhidden (+)= G . W[v0 : v0 + width]  (contraction over the chunk; long tiles first)
+    pr[count] = make_problem(n, h, gcols, false, true, kEpiAccumRows);
+    pr[count].b_k_off = int(v0);
+    ma[count] = t_g_k;
+    mb[count] = t_w_mn;
+    es.accum.acc32 = dh32;
+    es.accum.out = static_cast<__nv_bfloat16*>(dhidden);
+    es.accum.ld = h;
+    es.accum.rows = n;
+    es.accum.cols = h;
+    es.accum.mode = chunks == 1 ? 3 : (c == 0 ? 0 : (c == chunks - 1 ? 2 : 1));
     {
-      GemmShape g{};
-      g.m = width;
-      g.n = h;
-      g.k = n;
-      EpiStoreRows::Params ep{};
-      ep.out = static_cast<uint8_t*>(dweight) + size_t(v0) * h * wsz;
-      ep.ldo = h;
-      ep.rows = width;
-      ep.cols = h;
-      ep.f32 = w_dtype == FLCE_F32;
-      const double fl = 2.0 * double(n) * double(width) * double(h);
-      const double by = 2.0 * double(n) * (double(gcols) + double(h)) + double(wsz) * width * h;
-      if ((st = launch_gemm<EpiStoreRows, true, true>(t_g_mn, t_hid_mn, g, ep, *dev, cs,
-                                                      KF_GEMM_DW, fl, by)) != FLCE_OK)
-        return st;
+      const double rmw = es.accum.mode == 0 ? 4.0 : (es.accum.mode == 1 ? 8.0 : (es.accum.mode == 2 ? 6.0 : 2.0));
+      flops += 2.0 * double(n) * double(width) * double(h);
+      bytes += 2.0 * double(n) * gcols + 2.0 * double(width) * h + rmw * double(n) * h;
     }
-    // K5: dhidden (+)= G . W[v0 : v0 + width]  (contraction over the chunk).
-    {
-      GemmShape g{};
-      g.m = n;
-      g.n = h;
-      g.k = gcols;
-      g.b_k_off = int(v0);
-      EpiAccumRows::Params ep{};
-      ep.acc32 = dh32;
-      ep.out = static_cast<__nv_bfloat16*>(dhidden);
-      ep.ld = h;
-      ep.rows = n;
-      ep.cols = h;
-      ep.mode = chunks == 1 ? 3 : (c == 0 ? 0 : (c == chunks - 1 ? 2 : 1));
-      const double fl = 2.0 * double(n) * double(width) * double(h);
-      const double rmw = ep.mode == 0 ? 4.0 : (ep.mode == 1 ? 8.0 : (ep.mode == 2 ? 6.0 : 2.0));
-      const double by = 2.0 * double(n) * gcols + 2.0 * double(width) * h + rmw * double(n) * h;
-      if ((st = launch_gemm<EpiAccumRows, false, true>(t_g_k, t_w_mn, g, ep, *dev, cs,
-                                                       KF_GEMM_DH, fl, by)) != FLCE_OK)
-        return st;
+    ++count;
+    // K4: dW[v0 : v0 + width] = G^T . hidden  (contraction over tokens)
+    pr[count] = make_problem(width, h, n, true, true, kEpiStoreRows);
+    ma[count] = t_g_mn;
+    mb[count] = t_hid_mn;
+    es.store.out = static_cast<uint8_t*>(dweight) + size_t(v0) * h * wsz;
+    es.store.ldo = h;
+    es.store.rows = width;
+    es.store.cols = h;
+    es.store.f32 = w_dtype == FLCE_F32;
+    flops += 2.0 * double(n) * double(width) * double(h);
+    bytes += 2.0 * double(n) * (double(gcols) + double(h)) + double(wsz) * width * h;
+    ++count;
+    // K3 of the next chunk into the other G buffer
+    if (c + 1 < chunks) {
+      grad_problem(c + 1, &pr[count], &ma[count], &mb[count], &es.grad);
+      flops += grad_flops(c + 1);
+      bytes += grad_bytes(c + 1);
+      ++count;
     }
+    if ((st = launch_group<kEpiSetBackward, CfgDh, CfgDw, CfgGrad>(
+             pr, ma, mb, count, es, &counters[c + 1], *dev, cs, KF_GEMM_BWD, flops, bytes)) !=
+        FLCE_OK)
+      return st;
   }
   return FLCE_OK;
 }
@@ -795,11 +870,9 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   const bool ok_a = a_mn ? tmap_mnmajor(&ta, a, m, k, m) : tmap_kmajor(&ta, a, k, m, k, kBM);
   const bool ok_b = b_mn ? tmap_mnmajor(&tb, b, n, k, n) : tmap_kmajor(&tb, b, k, n, k, kBN);
   if (!ok_a || !ok_b) return FLCE_ERR_CUDA;
-  GemmShape g{};
-  g.m = m;
-  g.n = n;
-  g.k = k;
-  EpiStoreRows::Params ep{};
+  const GemmProblem prob = make_problem(m, n, k, a_mn != 0, b_mn != 0, kEpiStoreRows);
+  EpiSet<kEpiSetStore> es{};
+  EpiStoreRows::Params& ep = es.store;
   ep.out = d;
   ep.ldo = n;
   ep.rows = m;
@@ -809,12 +882,16 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   const double by = 2.0 * (double(m) + double(n)) * double(k) + 4.0 * double(m) * n;
   const int f = KF_SELFTEST_GEMM;
   if (!a_mn && !b_mn)
-    return launch_gemm<EpiStoreRows, false, false>(ta, tb, g, ep, *dev, cs, f, fl, by);
+    return launch_group<kEpiSetStore, ProblemCfg<false, false, kEpiStoreRows>>(
+        &prob, &ta, &tb, 1, es, nullptr, *dev, cs, f, fl, by);
   if (!a_mn && b_mn)
-    return launch_gemm<EpiStoreRows, false, true>(ta, tb, g, ep, *dev, cs, f, fl, by);
+    return launch_group<kEpiSetStore, ProblemCfg<false, true, kEpiStoreRows>>(
+        &prob, &ta, &tb, 1, es, nullptr, *dev, cs, f, fl, by);
   if (a_mn && !b_mn)
-    return launch_gemm<EpiStoreRows, true, false>(ta, tb, g, ep, *dev, cs, f, fl, by);
-  return launch_gemm<EpiStoreRows, true, true>(ta, tb, g, ep, *dev, cs, f, fl, by);
+    return launch_group<kEpiSetStore, ProblemCfg<true, false, kEpiStoreRows>>(
+        &prob, &ta, &tb, 1, es, nullptr, *dev, cs, f, fl, by);
+  return launch_group<kEpiSetStore, ProblemCfg<true, true, kEpiStoreRows>>(
+      &prob, &ta, &tb, 1, es, nullptr, *dev, cs, f, fl, by);
 }
 
 extern "C" int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream) {
