@@ -38,6 +38,7 @@
 #include "flce.h"
 #include "epilogues.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_sm100_pair.cuh"
 
 namespace flce {
 
@@ -51,6 +52,16 @@ constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1024;  // TMA coordinates are i
 constexpr size_t kAlign = 1024;
 constexpr size_t kChunkBudgetBytes = size_t(128) << 20;  // default size of each G buffer
 constexpr int64_t kMinChunk = 4096;
+
+// Contractions run on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2) unless
+// built with FLCE_SINGLE_CTA (one CTA per 128 x 256 tile).
+#ifdef FLCE_SINGLE_CTA
+constexpr bool kUsePairs = false;
+#else
+constexpr bool kUsePairs = true;
+#endif
+constexpr int kTileRows = kUsePairs ? kPairBM : kBM;      // output rows per tile
+constexpr int kBBoxRows = kUsePairs ? kBN / 2 : kBN;      // K-major B rows loaded per CTA
 
 // ------------------------------------------------------------------ kernels
 
@@ -386,10 +397,10 @@ constexpr int64_t kL2ResidentBytes = int64_t(40) << 20;
 
 static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
   TileRaster r{};
-  r.m_tiles = int(cdiv(m, kBM));
+  r.m_tiles = int(cdiv(m, kTileRows));
   r.n_tiles = int(cdiv(n, kBN));
   const int64_t kk = std::max<int64_t>(k, 1);
-  const int64_t a_panel = int64_t(kBM) * kk * 2, b_panel = int64_t(kBN) * kk * 2;
+  const int64_t a_panel = int64_t(kTileRows) * kk * 2, b_panel = int64_t(kBN) * kk * 2;
   const int64_t a_all = a_panel * r.m_tiles, b_all = b_panel * r.n_tiles;
   if (a_all <= kL2ResidentBytes && a_all <= b_all) {
     r.n_fast = 0;
@@ -443,13 +454,54 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   g.tile_counter = counter;
   g.err = dev.err;
   g.timeout_ns = kDefaultTimeoutNs;
-  auto kern = tc_gemm_group_kernel<EpiSet<kKinds>, C0, C1, C2>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(kGemmSmemBytes)) != cudaSuccess)
-    return FLCE_ERR_CUDA;
-  const int grid = int(std::min<int64_t>(dev.num_sms, total));
-  LaunchScope scope(family, flops, bytes, st);
-  kern<<<grid, kThreads, kGemmSmemBytes, st>>>(maps, g, ep);
+  if constexpr (kUsePairs) {
+    auto kern = tc_gemm_pair_kernel<EpiSet<kKinds>, C0, C1, C2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kPairSmemBytes)) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    // Pairs that can be resident at once (clusters need two SMs of one GPC).
+    static int max_pairs = 0;
+    if (max_pairs == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (dev.num_sms / 2), 1, 1);
+      q.blockDim = dim3(kThreads, 1, 1);
+      q.dynamicSmemBytes = kPairSmemBytes;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0)
+        n = dev.num_sms / 2;
+      max_pairs = std::min(n, dev.num_sms / 2);
+    }
+    const int pairs = int(std::min<int64_t>(max_pairs, total));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope scope(family, flops, bytes, st);
+    if (cudaLaunchKernelEx(&cfg, kern, maps, g, ep) != cudaSuccess) return FLCE_ERR_CUDA;
+  } else {
+    auto kern = tc_gemm_group_kernel<EpiSet<kKinds>, C0, C1, C2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kGemmSmemBytes)) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    const int grid = int(std::min<int64_t>(dev.num_sms, total));
+    LaunchScope scope(family, flops, bytes, st);
+    kern<<<grid, kThreads, kGemmSmemBytes, st>>>(maps, g, ep);
+  }
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -636,7 +688,7 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   }
 
   CUtensorMap ta, tb;
-  if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBN))
+  if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBBoxRows))
     return FLCE_ERR_CUDA;
   const GemmProblem prob = make_problem(n, v, h, false, false, kEpiForward);
   EpiSet<kEpiSetForward> es{};
@@ -736,7 +788,7 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
   CUtensorMap t_hid_k, t_w_k, t_hid_mn, t_w_mn;
-  if (!tmap_kmajor(&t_hid_k, hidden, h, n, h, kBM) || !tmap_kmajor(&t_w_k, wb, h, v, h, kBN) ||
+  if (!tmap_kmajor(&t_hid_k, hidden, h, n, h, kBM) || !tmap_kmajor(&t_w_k, wb, h, v, h, kBBoxRows) ||
       !tmap_mnmajor(&t_hid_mn, hidden, h, n, h) || !tmap_mnmajor(&t_w_mn, wb, h, v, h))
     return FLCE_ERR_CUDA;
 
@@ -868,7 +920,7 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? tmap_mnmajor(&ta, a, m, k, m) : tmap_kmajor(&ta, a, k, m, k, kBM);
-  const bool ok_b = b_mn ? tmap_mnmajor(&tb, b, n, k, n) : tmap_kmajor(&tb, b, k, n, k, kBN);
+  const bool ok_b = b_mn ? tmap_mnmajor(&tb, b, n, k, n) : tmap_kmajor(&tb, b, k, n, k, kBBoxRows);
   if (!ok_a || !ok_b) return FLCE_ERR_CUDA;
   const GemmProblem prob = make_problem(m, n, k, a_mn != 0, b_mn != 0, kEpiStoreRows);
   EpiSet<kEpiSetStore> es{};
