@@ -52,6 +52,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["flce", "chunked_ce"], default="flce",
+                    help="flce: the fused projection + CE (default); chunked_ce: cross entropy "
+                         "on given logits [4096, 128256] BF16")
     return ap.parse_args(argv)
 
 
@@ -453,8 +456,99 @@ def run_ours(args, w) -> int:
     return 0
 
 
+def run_chunked_ce(args) -> int:
+    """Cross entropy on given logits: forward + backward per step (HBM-bound)."""
+    import torch
+
+    from lm_head_projection_flce_b200 import flce
+    from lm_head_projection_flce_b200 import workloads as W
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device (sm_100a)")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    flce.load_library()
+    w = W.CE_LOGITS
+    d = W.generate_logits(w)
+    z = d["logits"].to(dev)
+    lab = d["labels"].to(dev)
+    n, v = z.shape
+    nlt = d["num_label_tokens"] if w.normalize_by_label_tokens else None
+    ws = torch.empty(int(flce.load_library().flce_ce_workspace_size(n)), dtype=torch.uint8,
+                     device=dev)
+    dz = torch.empty_like(z)
+    grad = torch.ones(1, device=dev)
+
+    def step(z_in=z, l_in=lab):
+        loss, lse = flce.ce_forward(z_in, l_in, reduction=w.reduction, num_label_tokens=nlt,
+                                    workspace=ws)
+        flce.ce_backward(z_in, l_in, lse, grad, reduction=w.reduction, num_label_tokens=nlt,
+                         dlogits=dz, workspace=ws)
+        return loss
+
+    warmup = max(args.warmup, 3)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    torch.cuda.synchronize(dev)
+    flce.profile_start()
+    l0 = flce.launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = flce.launch_count() - l0
+    stats = flce.profile_stop()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if flce.get_error(dev) != flce.FLCE_OK:
+        raise RuntimeError("device error word set during the timed region")
+    peaks, peak_src = load_peaks()
+    hbm = [k for k, st in stats.items() if st["bytes"] > 0 and k.startswith("ce_logits")]
+    dom_name = max(hbm, key=lambda k: stats[k]["total_ms"])
+    dom = stats[dom_name]
+    achieved = dom["bytes"] / (dom["total_ms"] / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": "cross entropy on given logits, fwd+bwd tokens/sec on 1 B200",
+        "value": n * args.steps / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "n_tokens": n, "vocab": v, "logits_dtype": w.dtype,
+                   "logits_sigma": w.sigma, "ignore_frac": w.ignore_frac,
+                   "reduction": "sum/num_label_tokens",
+                   "l2": "inputs larger than L2: 1.05 GB of logits read twice and 1.05 GB of "
+                         "gradient written every step"},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(w.name, dom_name),
+                     "bytes_per_launch": dom["bytes"] / dom["launches"],
+                     "peak_source": f"{peak_src} hbm_gbs (copy read+write)"},
+        "kernels": {k: {"launches_per_step": st["launches"] / args.steps,
+                        "ms_per_step": st["total_ms"] / args.steps,
+                        "gbs": st["bytes"] / (st["total_ms"] / 1e3) / 1e9 if st["total_ms"] > 0 else None}
+                    for k, st in sorted(stats.items())},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     args = parse_args(argv)
+    if args.path == "chunked_ce":
+        return run_chunked_ce(args)
     from lm_head_projection_flce_b200 import workloads as W
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":

@@ -158,6 +158,34 @@ int flce_selftest_gemm(const void* a, const void* b, float* d, int64_t m, int64_
 int flce_selftest_wait_timeout(unsigned int timeout_us, flce_stream_t stream);
 
 /*
+ * Cross entropy on given logits: the pages' ChunkedCrossEntropy
+ * ("nemo_automodel.components.loss.chunked_ce": ChunkedCrossEntropy.forward(
+ * logits, labels, mask, num_label_tokens), _ChunkedCrossEntropySum.forward /
+ * backward, compute_cross_entropy).
+ *   logits     [N, V] rows ld elements apart (ld >= V), BF16 (dtype 0) or FP32
+ *              (dtype 1), 16-byte aligned base; read, never written.
+ *   labels     int64 [N]; mask: optional uint8 [N] (NULL = none) -- a zero
+ *              entry makes that position ignored, as the page's `mask` does.
+ *   ignore_index, reduction, num_label_tokens, loss, lse: as flce_forward.
+ *   dlogits    (backward) [N, V], rows ld apart, the logits' dtype, 16-byte
+ *              aligned base: s_n * (softmax(logits)[n] - onehot(y_n)), zero
+ *              rows for ignored / masked positions.
+ *   workspace  >= flce_ce_workspace_size(N) bytes.
+ * No FP32 copy of the logits is made: one pass over them in the forward, one
+ * read + one write in the backward.  Same error conventions as flce_forward.
+ */
+size_t flce_ce_workspace_size(int64_t n_tokens);
+int flce_ce_forward(const void* logits, int dtype, const int64_t* labels, const uint8_t* mask,
+                    int64_t n_tokens, int64_t vocab, int64_t ld, int64_t ignore_index,
+                    int reduction, int64_t num_label_tokens, float* loss, float* lse,
+                    void* workspace, size_t ws_bytes, flce_stream_t stream);
+int flce_ce_backward(const void* logits, int dtype, const int64_t* labels, const uint8_t* mask,
+                     int64_t n_tokens, int64_t vocab, int64_t ld, int64_t ignore_index,
+                     int reduction, int64_t num_label_tokens, const float* grad_loss,
+                     const float* lse, void* dlogits, void* workspace, size_t ws_bytes,
+                     flce_stream_t stream);
+
+/*
  * Forward that allocates nothing and takes no workspace (the pages have no
  * counterpart; it exists for callers that cannot supply scratch memory, such
  * as a plugin inside a framework whose allocator owns the whole device, or a

@@ -39,6 +39,7 @@
 #include "epilogues.cuh"
 #include "gemm_sm100.cuh"
 #include "gemm_sm100_pair.cuh"
+#include "chunked_ce.cuh"
 
 namespace flce {
 
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kFinalThreads)
 // Backward prep (one block): valid-label count, per-token gradient scale
 // s_n = d loss / d token loss (0 for ignored / invalid labels), lse * log2(e).
 __global__ void __launch_bounds__(1024)
-    bwd_prep_kernel(const int64_t* __restrict__ labels, int64_t n_tokens, int64_t vocab,
+    bwd_prep_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
+                    int64_t n_tokens, int64_t vocab,
                     int64_t ignore_index, int reduction, int64_t num_label_tokens,
                     const float* __restrict__ grad_loss, const float* __restrict__ lse,
                     float* __restrict__ lse2, float* __restrict__ scale,
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(1024)
   bool bad = false;
   for (int64_t n = threadIdx.x; n < n_tokens; n += blockDim.x) {
     const int64_t y = labels[n];
-    if (y == ignore_index) continue;
+    if (y == ignore_index || (mask != nullptr && mask[n] == 0)) continue;
     if (y < 0 || y >= vocab) {
       bad = true;
       continue;
@@ -221,7 +223,8 @@ __global__ void __launch_bounds__(1024)
   }
   for (int64_t n = threadIdx.x; n < n_tokens; n += blockDim.x) {
     const int64_t y = labels[n];
-    const bool valid = y != ignore_index && y >= 0 && y < vocab;
+    const bool valid = y != ignore_index && (mask == nullptr || mask[n] != 0) && y >= 0 &&
+                       y < vocab;
     const float g = reduction == FLCE_NONE ? grad_loss[n] : base;
     scale[n] = valid ? g : 0.0f;
     lse2[n] = lse[n] * kLog2e;
@@ -301,12 +304,13 @@ static int device_info(DeviceInfo** out) {
 
 enum KernelFamily {
   KF_CAST = 0, KF_ZERO, KF_GEMM_FWD, KF_MERGE, KF_FINAL, KF_BWD_PREP, KF_GEMM_GRAD, KF_GEMM_DW,
-  KF_GEMM_DH, KF_SELFTEST_GEMM, KF_SELFTEST_WAIT, KF_GEMM_BWD, KF_COUNT
+  KF_GEMM_DH, KF_SELFTEST_GEMM, KF_SELFTEST_WAIT, KF_GEMM_BWD, KF_CE_FWD, KF_CE_BWD, KF_COUNT
 };
 static const char* const kFamilyNames[KF_COUNT] = {
     "cast_f32_bf16", "zero_rows",     "gemm_fwd_lse", "lse_merge",
     "loss_finalize", "bwd_prep",      "gemm_bwd_grad", "gemm_bwd_dw",
-    "gemm_bwd_dh",   "selftest_gemm", "selftest_wait", "gemm_bwd_fused"};
+    "gemm_bwd_dh",   "selftest_gemm", "selftest_wait", "gemm_bwd_fused",
+    "ce_logits_fwd", "ce_logits_bwd"};
 
 struct ProfRecord {
   int family;
@@ -781,7 +785,8 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
                              reinterpret_cast<__nv_bfloat16*>(ws + p.off_g) + size_t(n) * vc};
   {
     LaunchScope prep_scope(KF_BWD_PREP, 0.0, 24.0 * double(n), cs);
-    bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, n, v, ignore_index, reduction, num_label_tokens,
+    bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, nullptr, n, v, ignore_index, reduction,
+                                        num_label_tokens,
                                         grad_loss, lse, lse2, scale, counters,
                                         int(p.n_counters), dev->err);
   }
@@ -1064,4 +1069,133 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
   return flce_forward(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index, softcap,
                       reduction, num_label_tokens, loss, lse, scratch, kNoAllocScratchBytes,
                       stream);
+}
+
+// ===================================== cross entropy on given logits (chunked_ce)
+
+namespace flce {
+
+struct CePlan {
+  size_t off_loss, off_cnt, off_lse2, off_scale, total;
+};
+
+static CePlan plan_ce(int64_t n) {
+  CePlan p{};
+  size_t o = 0;
+  p.off_loss = o;  o = align_up(o + size_t(n) * 8);
+  p.off_cnt = o;   o = align_up(o + size_t(n) * 4);
+  p.off_lse2 = o;  o = align_up(o + size_t(n) * 4);
+  p.off_scale = o; o = align_up(o + size_t(n) * 4);
+  p.total = std::max(o, kAlign);
+  return p;
+}
+
+static int check_ce(const void* logits, int dtype, const int64_t* labels, int64_t n, int64_t v,
+                    int64_t ld, int reduction, int64_t num_label_tokens) {
+  if (n < 0 || v <= 0 || ld < v || n > kMaxDim || ld > (int64_t(1) << 40) / std::max<int64_t>(n, 1))
+    return FLCE_ERR_INVALID_ARG;
+  if (dtype != FLCE_BF16 && dtype != FLCE_F32) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_SUM && reduction != FLCE_MEAN && reduction != FLCE_NONE)
+    return FLCE_ERR_INVALID_ARG;
+  if (num_label_tokens > 0 && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  if (n > 0) {
+    if (logits == nullptr || labels == nullptr) return FLCE_ERR_INVALID_ARG;
+    if (!aligned(logits, 16) || !aligned(labels, 8)) return FLCE_ERR_INVALID_ARG;
+  }
+  return FLCE_OK;
+}
+
+static int ce_grid(const DeviceInfo& dev, int64_t n) {
+  return int(std::min<int64_t>(n, int64_t(dev.num_sms) * 16));
+}
+
+}  // namespace flce
+
+extern "C" size_t flce_ce_workspace_size(int64_t n_tokens) {
+  if (n_tokens < 0) return 0;
+  return plan_ce(n_tokens).total;
+}
+
+extern "C" int flce_ce_forward(const void* logits, int dtype, const int64_t* labels,
+                               const uint8_t* mask, int64_t n, int64_t v, int64_t ld,
+                               int64_t ignore_index, int reduction, int64_t num_label_tokens,
+                               float* loss, float* lse, void* workspace, size_t ws_bytes,
+                               flce_stream_t stream) {
+  int st = check_ce(logits, dtype, labels, n, v, ld, reduction, num_label_tokens);
+  if (st != FLCE_OK) return st;
+  if ((n > 0 || reduction != FLCE_NONE) && (loss == nullptr || !aligned(loss, 4)))
+    return FLCE_ERR_INVALID_ARG;
+  if (n > 0 && (lse == nullptr || !aligned(lse, 4))) return FLCE_ERR_INVALID_ARG;
+  const CePlan p = plan_ce(n);
+  if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p.total)
+    return FLCE_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* row_loss = reinterpret_cast<double*>(ws + p.off_loss);
+  int* row_cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  if (n > 0) {
+    const size_t esz = dtype == FLCE_F32 ? 4 : 2;
+    LaunchScope scope(KF_CE_FWD, 0.0, double(n) * double(v) * esz + 24.0 * double(n), cs);
+    float* tok = reduction == FLCE_NONE ? loss : nullptr;
+    if (dtype == FLCE_BF16)
+      ce_forward_kernel<__nv_bfloat16><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
+          static_cast<const __nv_bfloat16*>(logits), ld, labels, mask, n, v, ignore_index, lse,
+          tok, row_loss, row_cnt, dev->err);
+    else
+      ce_forward_kernel<float><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
+          static_cast<const float*>(logits), ld, labels, mask, n, v, ignore_index, lse, tok,
+          row_loss, row_cnt, dev->err);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  if (reduction != FLCE_NONE) {
+    LaunchScope scope(KF_FINAL, 0.0, 12.0 * double(n), cs);
+    loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(row_loss, row_cnt, int(n), reduction,
+                                                      num_label_tokens, loss);
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  return FLCE_OK;
+}
+
+extern "C" int flce_ce_backward(const void* logits, int dtype, const int64_t* labels,
+                                const uint8_t* mask, int64_t n, int64_t v, int64_t ld,
+                                int64_t ignore_index, int reduction, int64_t num_label_tokens,
+                                const float* grad_loss, const float* lse, void* dlogits,
+                                void* workspace, size_t ws_bytes, flce_stream_t stream) {
+  int st = check_ce(logits, dtype, labels, n, v, ld, reduction, num_label_tokens);
+  if (st != FLCE_OK) return st;
+  if (n > 0) {
+    if (grad_loss == nullptr || lse == nullptr || dlogits == nullptr) return FLCE_ERR_INVALID_ARG;
+    if (!aligned(grad_loss, 4) || !aligned(lse, 4) || !aligned(dlogits, 16))
+      return FLCE_ERR_INVALID_ARG;
+  }
+  const CePlan p = plan_ce(n);
+  if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p.total)
+    return FLCE_ERR_WORKSPACE;
+  if (n == 0) return FLCE_OK;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != FLCE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(ws + p.off_lse2);
+  float* scale = reinterpret_cast<float*>(ws + p.off_scale);
+  {
+    LaunchScope scope(KF_BWD_PREP, 0.0, 24.0 * double(n), cs);
+    bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, mask, n, v, ignore_index, reduction,
+                                        num_label_tokens, grad_loss, lse, lse2, scale, nullptr, 0,
+                                        dev->err);
+  }
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  const size_t esz = dtype == FLCE_F32 ? 4 : 2;
+  LaunchScope scope(KF_CE_BWD, 0.0, 2.0 * double(n) * double(v) * esz + 16.0 * double(n), cs);
+  if (dtype == FLCE_BF16)
+    ce_backward_kernel<__nv_bfloat16><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(logits), ld, labels, n, v, lse2, scale,
+        static_cast<__nv_bfloat16*>(dlogits));
+  else
+    ce_backward_kernel<float><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
+        static_cast<const float*>(logits), ld, labels, n, v, lse2, scale,
+        static_cast<float*>(dlogits));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }

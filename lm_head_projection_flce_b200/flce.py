@@ -59,6 +59,11 @@ SIGNATURES = {
     "flce_forward_noalloc": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64,
                                       _c_i64, _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr,
                                       _c_ptr, _c_ptr]),
+    "flce_ce_workspace_size": (_c_size, [_c_i64]),
+    "flce_ce_forward": (_c_int, [_c_ptr, _c_int, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
+                                 _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "flce_ce_backward": (_c_int, [_c_ptr, _c_int, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
+                                  _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_size, _c_ptr]),
     "flce_launch_count": (ctypes.c_ulonglong, []),
     "flce_profile_start": (_c_int, []),
     "flce_profile_stop": (_c_int, [_c_ptr, _c_int, ctypes.POINTER(_c_int)]),
@@ -301,3 +306,68 @@ def forward_noalloc(hidden, weight, labels, *, ignore_index: int = -100, softcap
                                   _stream_handle(dev, stream))
     _check("flce_forward_noalloc", st)
     return (loss if reduction == "none" else loss.reshape(())), lse
+
+
+# ---------------------------------------------------------------- cross entropy on given logits
+
+def _prepare_logits(logits, labels, mask):
+    if logits.dtype not in W_DTYPES:
+        raise TypeError("logits must be bf16 or fp32")
+    if labels.dtype != torch.int64:
+        raise TypeError("labels must be int64")
+    v = logits.shape[-1]
+    z = logits.reshape(-1, v)
+    lab = labels.reshape(-1)
+    if z.shape[0] != lab.shape[0]:
+        raise ValueError("logits and labels disagree on the number of tokens")
+    if z.stride(-1) != 1 or not lab.is_contiguous():
+        raise ValueError("logits rows and labels must be contiguous")
+    m = None
+    if mask is not None:
+        m = mask.reshape(-1).to(torch.uint8).contiguous()
+        if m.shape[0] != lab.shape[0]:
+            raise ValueError("mask must match labels")
+    for t in (z, lab) + ((m,) if m is not None else ()):
+        if t.device.type != "cuda" or t.device != z.device:
+            raise ValueError("tensors must be on one CUDA device")
+    return z, lab, m
+
+
+def ce_forward(logits, labels, *, mask=None, ignore_index: int = -100, reduction: str = "sum",
+               num_label_tokens: int | None = None, workspace=None, stream=None):
+    """Cross entropy of given logits [..., V] (ChunkedCrossEntropy).  Returns (loss, lse)."""
+    lib = load_library()
+    z, lab, m = _prepare_logits(logits, labels, mask)
+    n, v = z.shape
+    dev = z.device
+    loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
+    lse = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
+    st = lib.flce_ce_forward(_ptr(z), W_DTYPES[z.dtype], _ptr(lab), _ptr(m), n, v, z.stride(0),
+                             ignore_index, REDUCTIONS[reduction], int(num_label_tokens or 0),
+                             _ptr(loss), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(dev, stream))
+    _check("flce_ce_forward", st)
+    return (loss if reduction == "none" else loss.reshape(())), lse
+
+
+def ce_backward(logits, labels, lse, grad_loss, *, mask=None, ignore_index: int = -100,
+                reduction: str = "sum", num_label_tokens: int | None = None, dlogits=None,
+                workspace=None, stream=None):
+    """Gradient w.r.t. the logits, in the logits' dtype and shape."""
+    lib = load_library()
+    z, lab, m = _prepare_logits(logits, labels, mask)
+    n, v = z.shape
+    dev = z.device
+    grad = grad_loss.reshape(-1).to(device=dev, dtype=torch.float32).contiguous()
+    if dlogits is None:
+        dlogits = torch.empty_like(z)
+    out = dlogits.reshape(n, v)
+    if out.stride(0) != z.stride(0) or out.stride(1) != 1:
+        raise ValueError("dlogits must have the logits' row stride")
+    ws = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
+    st = lib.flce_ce_backward(_ptr(z), W_DTYPES[z.dtype], _ptr(lab), _ptr(m), n, v, z.stride(0),
+                              ignore_index, REDUCTIONS[reduction], int(num_label_tokens or 0),
+                              _ptr(grad), _ptr(lse), _ptr(out), _ptr(ws), ws.numel(),
+                              _stream_handle(dev, stream))
+    _check("flce_ce_backward", st)
+    return out.reshape(logits.shape)

@@ -160,3 +160,36 @@ def generate(w: Workload, device: str | torch.device = "cpu") -> dict:
     if str(device) != "cpu":
         out = {k_: (t.to(device) if isinstance(t, torch.Tensor) else t) for k_, t in out.items()}
     return out
+
+
+# Cross entropy on given logits (the chunked_ce page's ChunkedCrossEntropy):
+# logits [N, V] in BF16 drawn N(0, sigma) with sigma = 1.28, the spread of the
+# logits of the 4096 x 4096 x 128256 workload (hidden N(0,1), head N(0, 0.02):
+# std = 0.02 * sqrt(4096)); labels uniform, 5% ignored.
+@dataclasses.dataclass(frozen=True)
+class LogitsWorkload:
+    name: str
+    n_tokens: int
+    vocab: int
+    dtype: str = "bf16"
+    sigma: float = 1.28
+    ignore_frac: float = 0.05
+    reduction: str = "sum"
+    normalize_by_label_tokens: bool = True
+    seed: int = 0
+
+
+CE_LOGITS = LogitsWorkload(name="ce_logits_n4096_v128256_bf16", n_tokens=4096, vocab=128256,
+                           seed=3002)
+
+
+def generate_logits(w: LogitsWorkload) -> dict:
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    logits = torch.randn(w.n_tokens, w.vocab, generator=g, dtype=torch.float32).mul_(w.sigma)
+    logits = logits.to(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+    labels = torch.randint(0, w.vocab, (w.n_tokens,), generator=g, dtype=torch.int64)
+    k = int(math.floor(w.ignore_frac * w.n_tokens + 0.5))
+    if k > 0:
+        labels[torch.randperm(w.n_tokens, generator=g)[:k]] = IGNORE_INDEX
+    return {"logits": logits, "labels": labels,
+            "num_label_tokens": int((labels != IGNORE_INDEX).sum().item())}

@@ -46,7 +46,7 @@ __all__ = [
     "bf16_round", "compute_head", "project", "apply_softcap", "logsumexp_rows",
     "token_losses", "reduce_losses", "token_scales", "logit_grad",
     "ForwardResult", "forward", "backward", "forward_rows", "dh_rows", "dw_rows",
-    "check_labels",
+    "check_labels", "ce_labels", "ce_forward", "ce_backward",
 ]
 
 
@@ -299,3 +299,41 @@ def dw_rows(hidden, weight, labels, vrows, lse_all, *, ignore_index=-100, softca
     g *= s[:, None]
     out[live] = g.T @ np.asarray(hidden, dtype=np.float64)
     return out
+
+
+# --------------------------------------------------------------------------
+# Cross entropy on given logits ("nemo_automodel.components.loss.chunked_ce":
+# ChunkedCrossEntropy.forward, _ChunkedCrossEntropySum.forward/backward)
+# --------------------------------------------------------------------------
+
+def ce_labels(labels, mask, ignore_index: int = -100) -> np.ndarray:
+    """Labels with every position whose mask is zero replaced by ``ignore_index``
+    (ChunkedCrossEntropy.forward, parameter ``mask``: nonzero positions
+    contribute, zero positions are ignored)."""
+    labels = np.array(labels, dtype=np.int64, copy=True)
+    if mask is not None:
+        labels[np.asarray(mask) == 0] = ignore_index
+    return labels
+
+
+def ce_forward(logits, labels, *, mask=None, ignore_index: int = -100,
+               reduction: str = "sum", num_label_tokens: int | None = None) -> ForwardResult:
+    """Cross entropy of given logits ``[N, V]`` (any float dtype, upcast to FP64)."""
+    z = np.asarray(logits, dtype=np.float64)
+    lab = ce_labels(labels, mask, ignore_index)
+    valid = check_labels(lab, z.shape[1], ignore_index)
+    lse = logsumexp_rows(z) if z.shape[0] else np.zeros(0)
+    tok = token_losses(lse, z, lab, valid)
+    return ForwardResult(reduce_losses(tok, valid, reduction, num_label_tokens), lse, tok)
+
+
+def ce_backward(logits, labels, *, mask=None, ignore_index: int = -100,
+                reduction: str = "sum", num_label_tokens: int | None = None,
+                grad_loss=1.0) -> np.ndarray:
+    """Gradient of that loss w.r.t. the logits (_ChunkedCrossEntropySum.backward)."""
+    z = np.asarray(logits, dtype=np.float64)
+    lab = ce_labels(labels, mask, ignore_index)
+    valid = check_labels(lab, z.shape[1], ignore_index)
+    lse = logsumexp_rows(z) if z.shape[0] else np.zeros(0)
+    s = token_scales(valid, reduction, num_label_tokens, grad_loss)
+    return logit_grad(z, lse, lab, valid, s, 0.0)

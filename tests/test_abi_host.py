@@ -164,3 +164,31 @@ def test_binding_refuses_cpu_tensors():
         flce.forward(h, w, y)
     with pytest.raises(TypeError):
         flce.forward(h.float(), w, y)
+
+
+def test_ce_entry_points_fail_closed_on_the_host(lib):
+    def fwd(**kw):
+        a = dict(z=FAKE, dt=0, lab=FAKE, mask=None, n=64, v=1000, ld=1000, ii=-100, red=0, nlt=0,
+                 loss=FAKE, lse=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return lib.flce_ce_forward(a["z"], a["dt"], a["lab"], a["mask"], a["n"], a["v"], a["ld"],
+                                   a["ii"], a["red"], a["nlt"], a["loss"], a["lse"], a["ws"],
+                                   a["wsb"], None)
+
+    def bwd(**kw):
+        a = dict(z=FAKE, dt=1, lab=FAKE, mask=None, n=64, v=1000, ld=1000, ii=-100, red=0, nlt=0,
+                 g=FAKE, lse=FAKE, dz=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return lib.flce_ce_backward(a["z"], a["dt"], a["lab"], a["mask"], a["n"], a["v"], a["ld"],
+                                    a["ii"], a["red"], a["nlt"], a["g"], a["lse"], a["dz"], a["ws"],
+                                    a["wsb"], None)
+
+    for call in (fwd, bwd):
+        for kw in (dict(v=0), dict(ld=999), dict(n=-1), dict(dt=5), dict(red=7),
+                   dict(red=1, nlt=3), dict(z=0), dict(lab=0), dict(z=FAKE + 4), dict(lab=FAKE + 2)):
+            assert call(**kw) == 1, (call.__name__, kw)
+        assert call(ws=0) == 2 and call(wsb=10) == 2
+    for kw in (dict(g=0), dict(lse=0), dict(dz=0), dict(dz=FAKE + 8)):
+        assert bwd(**kw) == 1, kw
+    assert fwd(loss=0) == 1 and fwd(lse=0) == 1
+    assert lib.flce_ce_workspace_size(4096) >= 4096 * 20 and lib.flce_ce_workspace_size(-1) == 0

@@ -1,0 +1,138 @@
+"""GPU parity of cross entropy on given logits (the chunked_ce page's
+ChunkedCrossEntropy) against the FP64 oracle: BF16 and FP32 logits, rows that
+do not start on a 16-byte boundary, row strides, masks, every reduction and
+the edge cases.  Tolerances as for the fused path: |dlse| <= 2e-3, loss
+relative error <= 1e-4, max|d dlogits| <= 1e-2 * max|ref|."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_projection_flce_b200 import flce
+from oracle import flce_oracle as O
+
+from gpu_common import GRAD_REL, LOSS_REL, LSE_ABS, gpu_device, max_rel
+
+pytestmark = pytest.mark.gpu
+II = -100
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return gpu_device()
+
+
+def _case(seed, n, v, dtype, ignore_frac=0.1, scale=2.0, ld=None):
+    g = torch.Generator().manual_seed(seed)
+    ld = v if ld is None else ld
+    full = (torch.randn(n, ld, generator=g) * scale).to(dtype)
+    logits = full[:, :v]
+    labels = torch.randint(0, v, (n,), generator=g)
+    k = int(math.floor(ignore_frac * n + 0.5))
+    if k:
+        labels[torch.randperm(n, generator=g)[:k]] = II
+    return full, logits, labels
+
+
+def _check(dev, logits, labels, *, mask=None, reduction="sum", nlt=None, grad=None):
+    z = logits.to(dev)
+    lab = labels.to(dev)
+    m = None if mask is None else mask.to(dev)
+    loss, lse = flce.ce_forward(z, lab, mask=m, reduction=reduction, num_label_tokens=nlt)
+    if grad is None:
+        grad = torch.ones(1) if reduction != "none" else torch.ones(labels.shape[0])
+    dz = flce.ce_backward(z, lab, lse, grad.to(dev), mask=m, reduction=reduction,
+                          num_label_tokens=nlt)
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
+    zf = logits.double().numpy()
+    mk = None if mask is None else mask.numpy()
+    ref = O.ce_forward(zf, labels.numpy(), mask=mk, reduction=reduction, num_label_tokens=nlt)
+    rdz = O.ce_backward(zf, labels.numpy(), mask=mk, reduction=reduction, num_label_tokens=nlt,
+                        grad_loss=grad.double().numpy())
+    assert float(np.max(np.abs(lse.double().cpu().numpy() - ref.lse))) <= LSE_ABS
+    lg = np.asarray(loss.double().cpu().numpy()).reshape(-1)
+    lr = np.asarray(ref.loss).reshape(-1)
+    if lr.size == 1:
+        if math.isnan(lr[0]):
+            assert math.isnan(lg[0])
+        elif lr[0] == 0:
+            assert lg[0] == 0
+        else:
+            assert abs(lg[0] - lr[0]) <= LOSS_REL * abs(lr[0])
+    else:
+        assert float(np.max(np.abs(lg - lr))) <= LSE_ABS
+    assert dz.dtype == logits.dtype and dz.shape == logits.shape
+    assert max_rel(dz.double().cpu().numpy(), rdz) <= GRAD_REL
+    return dz
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("n,v", [(64, 1024), (333, 1000), (129, 12289), (8, 7), (300, 50001)])
+def test_ce_parity(dev, dtype, n, v):
+    _, logits, labels = _case(n * 31 + v, n, v, dtype)
+    _check(dev, logits, labels)
+
+
+@pytest.mark.parametrize("reduction,nlt", [("mean", None), ("none", None), ("sum", 77)])
+def test_ce_reductions_and_mask(dev, reduction, nlt):
+    _, logits, labels = _case(5, 257, 3001, torch.bfloat16)
+    mask = (torch.arange(257) % 5 != 0).to(torch.uint8)
+    grad = torch.linspace(-1, 2, 257) if reduction == "none" else torch.tensor([1.5])
+    dz = _check(dev, logits, labels, mask=mask, reduction=reduction, nlt=nlt, grad=grad)
+    assert torch.all(dz[::5] == 0)
+
+
+def test_ce_row_stride_and_unaligned_rows(dev):
+    # rows 1001 elements apart: every row starts at a different 16-byte phase
+    full, logits, labels = _case(6, 90, 997, torch.bfloat16, ld=1001)
+    z = full.to(dev)[:, :997]
+    lab = labels.to(dev)
+    loss, lse = flce.ce_forward(z, lab)
+    dbuf = torch.full((90, 1001), 7.0, dtype=torch.bfloat16, device=dev)
+    flce.ce_backward(z, lab, lse, torch.ones(1, device=dev), dlogits=dbuf[:, :997])
+    torch.cuda.synchronize(dev)
+    ref = O.ce_forward(logits.double().numpy(), labels.numpy())
+    rdz = O.ce_backward(logits.double().numpy(), labels.numpy())
+    assert float(np.max(np.abs(lse.double().cpu().numpy() - ref.lse))) <= LSE_ABS
+    assert max_rel(dbuf[:, :997].double().cpu().numpy(), rdz) <= GRAD_REL
+    assert torch.all(dbuf[:, 997:] == 7.0)          # the gap between rows is untouched
+
+
+def test_ce_edge_cases(dev):
+    z = torch.zeros(0, 50, dtype=torch.bfloat16, device=dev)
+    lab = torch.zeros(0, dtype=torch.int64, device=dev)
+    loss, _ = flce.ce_forward(z, lab)
+    mean, _ = flce.ce_forward(z, lab, reduction="mean")
+    torch.cuda.synchronize(dev)
+    assert float(loss) == 0.0 and math.isnan(float(mean))
+    _, logits, labels = _case(8, 40, 300, torch.float32, ignore_frac=1.0)
+    dz = _check(dev, logits, labels)
+    assert torch.all(dz == 0)
+    # a bad label is flagged and contributes nothing
+    _, logits, labels = _case(9, 40, 300, torch.bfloat16, ignore_frac=0.0)
+    bad = labels.clone()
+    bad[4] = 300
+    zz = logits.to(dev)
+    loss, lse = flce.ce_forward(zz, bad.to(dev))
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_ERR_BAD_LABEL
+    fixed = bad.clone()
+    fixed[4] = II
+    ref = O.ce_forward(logits.double().numpy(), fixed.numpy())
+    assert abs(float(loss) - ref.loss) <= LOSS_REL * abs(ref.loss)
+
+
+def test_ce_matches_fused_path_on_materialised_logits(dev):
+    """The fused projection + CE equals CE on the FP32 logits it never writes."""
+    g = torch.Generator().manual_seed(10)
+    hid = torch.randn(200, 256, generator=g).to(torch.bfloat16).to(dev)
+    wt = (torch.randn(3000, 256, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+    lab = torch.randint(0, 3000, (200,), generator=g).to(dev)
+    l1, lse1 = flce.forward(hid, wt, lab)
+    logits = hid.float() @ wt.float().T
+    l2, lse2 = flce.ce_forward(logits, lab)
+    torch.cuda.synchronize(dev)
+    assert torch.allclose(lse1, lse2, atol=1e-3, rtol=0)
+    assert abs(float(l1) - float(l2)) <= 1e-4 * abs(float(l2))

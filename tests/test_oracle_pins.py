@@ -424,3 +424,44 @@ def test_pins_catch_planted_mistakes(mutant, monkeypatch):
         except (AssertionError, ValueError, IndexError, FloatingPointError):
             caught.append(pin.__name__)
     assert caught, f"no pin detects: {mutant}"
+
+
+# ---------------------------------------------------------------------------
+# Cross entropy on given logits (chunked_ce page)
+# ---------------------------------------------------------------------------
+
+def test_ce_oracle_matches_torch_cross_entropy():
+    """Forward and logits gradient equal torch's cross_entropy and its autograd
+    on FP64 logits, with ignore_index, mask and every reduction."""
+    rng = np.random.default_rng(21)
+    n, v = 11, 37
+    z = rng.standard_normal((n, v)) * 2.0
+    labels = rng.integers(0, v, size=n)
+    labels[3] = II
+    mask = np.ones(n, dtype=np.uint8)
+    mask[[0, 7]] = 0
+    eff = labels.copy()
+    eff[[0, 7]] = II
+    g = np.linspace(0.5, 1.5, n)
+    for red, nlt, grad in (("sum", None, 1.3), ("sum", 6, 0.7), ("mean", None, 2.0), ("none", None, g)):
+        r = O.ce_forward(z, labels, mask=mask, reduction=red, num_label_tokens=nlt)
+        zt = torch.tensor(z, requires_grad=True)
+        loss = F.cross_entropy(zt, torch.from_numpy(eff), ignore_index=II, reduction=red)
+        if nlt is not None:
+            loss = loss / nlt
+        assert np.allclose(r.loss, loss.detach().numpy(), rtol=1e-13, atol=1e-13)
+        loss.backward(torch.as_tensor(grad, dtype=torch.float64).reshape(loss.shape))
+        dz = O.ce_backward(z, labels, mask=mask, reduction=red, num_label_tokens=nlt, grad_loss=grad)
+        assert np.allclose(dz, zt.grad.numpy(), rtol=1e-12, atol=1e-14)
+    assert np.all(O.ce_backward(z, labels, mask=mask)[[0, 3, 7]] == 0.0)
+
+
+def test_ce_oracle_equals_fused_oracle_with_identity_head():
+    """With W = I the fused loss is the cross entropy of the hidden values."""
+    rng = np.random.default_rng(22)
+    n, v = 6, 9
+    h = _bf16_vals(rng, (n, v), 1.7)
+    labels = rng.integers(0, v, size=n)
+    a = O.ce_forward(h, labels)
+    b = O.forward(h, np.eye(v), labels)
+    assert abs(a.loss - b.loss) < 1e-12 and np.allclose(a.lse, b.lse, atol=1e-13)
