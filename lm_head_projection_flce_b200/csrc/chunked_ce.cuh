@@ -93,8 +93,34 @@ __global__ void __launch_bounds__(kCeThreads)
     for (int64_t i = threadIdx.x; i < head; i += kCeThreads)
       ms_merge(m, s, CeVec<T>::one(row + i) * kLog2e, 1.0f);
     const T* body = row + head;
-#pragma unroll 2
-    for (int64_t j = threadIdx.x; j < nvec; j += kCeThreads) {
+    // Four independent 16-byte loads in flight per thread, then one rescale.
+    constexpr int U = 4;
+    int64_t j = threadIdx.x;
+    for (; j + (U - 1) * kCeThreads < nvec; j += U * kCeThreads) {
+      float x[U][VN];
+#pragma unroll
+      for (int u = 0; u < U; ++u) CeVec<T>::load(body + (j + u * kCeThreads) * VN, x[u]);
+      float vm = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int e = 0; e < VN; ++e) {
+          x[u][e] *= kLog2e;
+          vm = fmaxf(vm, x[u][e]);
+        }
+      if (vm == -INFINITY) continue;
+      if (vm > m) {
+        s = s * fast_exp2(m - vm);
+        m = vm;
+      }
+      float acc = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int e = 0; e < VN; ++e) acc += fast_exp2(x[u][e] - m);
+      s += acc;
+    }
+    for (; j < nvec; j += kCeThreads) {
       float x[VN];
       CeVec<T>::load(body + j * VN, x);
       float vm = -INFINITY;
