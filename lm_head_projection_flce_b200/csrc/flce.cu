@@ -51,7 +51,7 @@ constexpr int kMergeWarps = 8;
 constexpr int kFinalThreads = 256;
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1024;  // TMA coordinates are int32
 constexpr size_t kAlign = 1024;
-constexpr size_t kChunkBudgetBytes = size_t(128) << 20;  // default size of each G buffer
+constexpr size_t kChunkBudgetBytes = size_t(1) << 30;  // default cap on each G buffer
 constexpr int64_t kMinChunk = 4096;
 
 // Contractions run on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2) unless
@@ -563,7 +563,7 @@ static FwdPlan plan_forward(const Shape& s) {
 }
 
 static int64_t default_chunk(const Shape& s) {
-  const int64_t cap = cdiv(cdiv(s.v, 4), kBN) * kBN;  // at most a quarter of the vocabulary
+  const int64_t cap = cdiv(cdiv(s.v, 6), kBN) * kBN;  // at most a sixth of the vocabulary
   int64_t budget = int64_t(kChunkBudgetBytes / (2 * size_t(std::max<int64_t>(s.n, 1))));
   budget = budget / kBN * kBN;
   return std::max<int64_t>(kBN, std::min(cap, std::max(kMinChunk, budget)));

@@ -239,3 +239,17 @@ def test_results_are_bitwise_reproducible(dev):
     for other in outs[1:]:
         for a, b in zip(outs[0], other):
             assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("softcap", [1.0, 30.0])
+def test_softcap_saturates_on_huge_logits(dev, softcap):
+    """Logits of +-1e3 and beyond: the capped logits sit at +-c, so every lse
+    lies in [-c + log V, c + log V], and gradients stay finite and match the oracle."""
+    w = W.custom(160, 64, 700, 704, softcap=softcap, ignore_frac=0.1, w_sigma=40.0, seed=24)
+    d = W.generate(w)
+    got = run_gpu(d, w, dev)
+    ref = run_oracle(d, w)
+    assert np.all(np.isfinite(got["dh"])) and np.all(np.isfinite(got["dw"]))
+    lo, hi = -softcap + np.log(700) - 1e-3, softcap + np.log(700) + 1e-3
+    assert np.all(got["lse"] >= lo) and np.all(got["lse"] <= hi)
+    assert_parity(got, ref)
