@@ -253,6 +253,7 @@ struct DeviceInfo {
   bool init = false;
   int status = FLCE_OK;
   int num_sms = 0;
+  int max_pairs = 0;  // CTA pairs of the pair GEMM that fit at once (0 = not yet queried)
   unsigned* err = nullptr;
 };
 
@@ -463,8 +464,9 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kPairSmemBytes)) != cudaSuccess)
       return FLCE_ERR_CUDA;
-    // Pairs that can be resident at once (clusters need two SMs of one GPC).
-    static int max_pairs = 0;
+    // Pairs that can be resident at once (clusters need two SMs of one GPC);
+    // queried once per device (every instantiation shares the launch shape).
+    int max_pairs = dev.max_pairs;
     if (max_pairs == 0) {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(2 * (dev.num_sms / 2), 1, 1);
@@ -481,6 +483,8 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
       if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0)
         n = dev.num_sms / 2;
       max_pairs = std::min(n, dev.num_sms / 2);
+      std::lock_guard<std::mutex> lock(g_mutex);
+      const_cast<DeviceInfo&>(dev).max_pairs = max_pairs;
     }
     const int pairs = int(std::min<int64_t>(max_pairs, total));
     cudaLaunchConfig_t cfg = {};

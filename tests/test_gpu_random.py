@@ -1,0 +1,73 @@
+"""Randomised GPU parity sweep: shapes (ragged in N, H, V and Vp), head dtype,
+softcap, reduction, num_label_tokens, ignore_index values (including one that
+is a large positive number), ignored fraction and workspace size (hence the
+backward's vocabulary chunking), each against the FP64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from lm_head_projection_flce_b200 import flce
+from lm_head_projection_flce_b200 import workloads as W
+from oracle import flce_oracle as O
+
+from gpu_common import assert_parity, gpu_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return gpu_device()
+
+
+def _draw(i):
+    r = np.random.default_rng(500 + i)
+    n = int(r.integers(1, 700))
+    h = int(8 * r.integers(1, 80))
+    v = int(r.integers(1, 4000))
+    vp = v + int(r.integers(0, 3)) * int(r.integers(0, 300))
+    return dict(n=n, h=h, v=v, vp=vp,
+                w_dtype=str(r.choice(["bf16", "f32"])),
+                softcap=float(r.choice([0.0, 0.0, 5.0, 30.0])),
+                reduction=str(r.choice(["sum", "sum", "mean", "none"])),
+                norm=bool(r.integers(0, 2)),
+                ignore_index=int(r.choice([-100, -1, 10 ** 6])),
+                ignore_frac=float(r.choice([0.0, 0.1, 0.5])),
+                ws_frac=float(r.choice([0.0, 0.5, 1.0])),
+                w_sigma=float(r.choice([0.02, 0.1])),
+                seed=600 + i)
+
+
+@pytest.mark.parametrize("i", range(24))
+def test_random_case(dev, i):
+    c = _draw(i)
+    w = W.custom(c["n"], c["h"], c["v"], c["vp"], w_dtype=c["w_dtype"], softcap=c["softcap"],
+                 ignore_frac=c["ignore_frac"], w_sigma=c["w_sigma"], seed=c["seed"])
+    d = W.generate(w)
+    labels = d["labels"].clone()
+    labels[labels == W.IGNORE_INDEX] = c["ignore_index"]
+    red = c["reduction"]
+    nlt = d["num_label_tokens"] if (red == "sum" and c["norm"] and d["num_label_tokens"] > 0) else None
+    wdt = torch.float32 if c["w_dtype"] == "f32" else torch.bfloat16
+    lo = flce.workspace_size(c["n"], c["h"], c["vp"], c["v"], wdt, minimum=True)
+    hi = flce.workspace_size(c["n"], c["h"], c["vp"], c["v"], wdt)
+    ws_bytes = int(lo + c["ws_frac"] * (hi - lo))
+    hid, wt, lab = d["hidden"].to(dev), d["weight"].to(dev), labels.to(dev)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    grad = torch.linspace(-1, 1, c["n"]) if red == "none" else torch.tensor([1.25])
+    loss, lse = flce.forward(hid, wt, lab, ignore_index=c["ignore_index"], softcap=c["softcap"],
+                             unpadded_vocab=c["v"], reduction=red, num_label_tokens=nlt, workspace=ws)
+    dh, dw = flce.backward(hid, wt, lab, lse, grad.to(dev), ignore_index=c["ignore_index"],
+                           softcap=c["softcap"], unpadded_vocab=c["v"], reduction=red,
+                           num_label_tokens=nlt, workspace=ws)
+    torch.cuda.synchronize(dev)
+    got = {"loss": loss.double().cpu().numpy(), "lse": lse.double().cpu().numpy(),
+           "dh": dh.double().cpu().numpy(), "dw": dw.double().cpu().numpy(),
+           "status": flce.get_error(dev)}
+    hw = d["weight"].numpy() if wdt == torch.float32 else d["weight"].double().numpy()
+    kw = dict(ignore_index=c["ignore_index"], softcap=c["softcap"], unpadded_vocab=c["v"],
+              reduction=red, num_label_tokens=nlt)
+    fwd = O.forward(d["hidden"].double().numpy(), hw, labels.numpy(), **kw)
+    rdh, rdw = O.backward(d["hidden"].double().numpy(), hw, labels.numpy(),
+                          grad_loss=grad.double().numpy(), **kw)
+    assert_parity(got, {"loss": np.asarray(fwd.loss), "lse": fwd.lse, "dh": rdh, "dw": rdw}), c
