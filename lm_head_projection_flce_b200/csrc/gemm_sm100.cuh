@@ -217,7 +217,6 @@ __device__ __forceinline__ bool mma_tile(int num_kb, uint32_t d_tmem, uint32_t s
   const uint64_t b_desc0 = b_hi | static_cast<uint64_t>(((smem_base + kATileBytes) & 0x3FFFFu) >> 4);
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_phase(bar_base + 8u * stage, phase, ctl, g.err, g.timeout_ns)) return false;
-    tc_fence_after_sync();
     const uint64_t soff = static_cast<uint64_t>((stage * kStageBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < kBK / kUmmaK; ++kk)

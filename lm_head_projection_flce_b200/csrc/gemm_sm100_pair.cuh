@@ -87,7 +87,6 @@ __device__ __forceinline__ bool pair_mma_tile(int num_kb, uint32_t d_tmem, uint3
       b_hi | static_cast<uint64_t>(((smem_base + kPairATileBytes) & 0x3FFFFu) >> 4);
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_phase(bar_base + 8u * stage, phase, ctl, g.err, g.timeout_ns)) return false;
-    tc_fence_after_sync();
     const uint64_t soff = static_cast<uint64_t>((stage * kPairStageBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < kBK / kUmmaK; ++kk)
@@ -186,16 +185,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t next_static = pair_id;
       const uint32_t sched_addr = smem_u32(sched_tile);
       const uint32_t peer_sched_addr = map_shared_to_rank(sched_addr, 1);
+      // The leader claims one tile ahead, so the counter's round trip overlaps
+      // the current tile's loads.
+      auto claim = [&]() -> int64_t {
+        int64_t c;
+        if (g.tile_counter != nullptr)
+          c = static_cast<int64_t>(atomicAdd(g.tile_counter, 1u));
+        else {
+          c = next_static;
+          next_static += num_pairs;
+        }
+        return c >= g.total_tiles ? -1 : c;
+      };
+      int64_t claimed = rank == 0 ? claim() : -1;
       while (ok) {
         int64_t t;
         if (rank == 0) {
-          if (g.tile_counter != nullptr)
-            t = static_cast<int64_t>(atomicAdd(g.tile_counter, 1u));
-          else {
-            t = next_static;
-            next_static += num_pairs;
-          }
-          if (t >= g.total_tiles) t = -1;
+          t = claimed;
           if (!wait_phase(bar_base + sempty_off(slot), sphase ^ 1u, ctl, g.err, g.timeout_ns)) {
             ok = false;
             break;
@@ -216,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sphase ^= 1u;
         }
         if (t < 0) break;
+        if (rank == 0) claimed = claim();
         const int p = problem_of(g, t);
         const GemmProblem& pr = g.prob[p];
         int mt, nt;
