@@ -455,6 +455,7 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   }
   g.num_problems = count;
   if (total == 0) return FLCE_OK;
+  if (total >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;  // the tile counter is 32-bit
   g.total_tiles = total;
   g.tile_counter = counter;
   g.err = dev.err;
