@@ -29,7 +29,13 @@
  *    aligned; labels, loss and lse 8- resp. 4-byte aligned.
  *  - Arguments are checked on the host before anything is enqueued; a bad
  *    argument returns an error status and enqueues nothing.  Nothing throws or
- *    aborts across this boundary.
+ *    aborts across this boundary.  FLCE_ERR_CUDA from a launch means kernels
+ *    the call enqueued before it may still run; the call's outputs are then
+ *    undefined.
+ *  - After one call per device (which queries the device and resolves the
+ *    tensor-map encoder), flce_forward / flce_backward / flce_ce_* only
+ *    enqueue kernels on `stream`, so a sequence of them can be captured into
+ *    a CUDA graph and replayed with the same buffers.
  *  - Labels outside [0, V) that are not ignore_index cannot be checked on the
  *    host without a device read; the kernels treat them as ignored (zero loss,
  *    zero gradient) and raise FLCE_ERR_BAD_LABEL in a per-device error word
@@ -51,7 +57,7 @@ typedef enum {
   FLCE_OK = 0,
   FLCE_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or option        */
   FLCE_ERR_WORKSPACE = 2,   /* workspace NULL or smaller than required       */
-  FLCE_ERR_UNSUPPORTED = 3, /* no sm_100a device / too large for this build  */
+  FLCE_ERR_UNSUPPORTED = 3, /* no sm_100a device, or more tiles than supported */
   FLCE_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed   */
   FLCE_ERR_BAD_LABEL = 5,   /* (flce_get_error) a label outside [0,V) seen   */
   FLCE_ERR_TIMEOUT = 6      /* (flce_get_error) a pipeline wait ran out      */

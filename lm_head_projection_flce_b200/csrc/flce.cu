@@ -441,7 +441,7 @@ static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool
 template <int kKinds, class C0, class C1 = NoProblem, class C2 = NoProblem>
 static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
                         const CUtensorMap* maps_b, int count, const EpiSet<kKinds>& ep,
-                        unsigned* counter, const DeviceInfo& dev, cudaStream_t st, int family,
+                        unsigned* counter, DeviceInfo& dev, cudaStream_t st, int family,
                         double flops, double bytes) {
   GemmMaps maps;
   GemmGroup g{};
@@ -485,7 +485,7 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
         n = dev.num_sms / 2;
       max_pairs = std::min(n, dev.num_sms / 2);
       std::lock_guard<std::mutex> lock(g_mutex);
-      const_cast<DeviceInfo&>(dev).max_pairs = max_pairs;
+      dev.max_pairs = max_pairs;
     }
     const int pairs = int(std::min<int64_t>(max_pairs, total));
     cudaLaunchConfig_t cfg = {};

@@ -253,3 +253,43 @@ def test_softcap_saturates_on_huge_logits(dev, softcap):
     lo, hi = -softcap + np.log(700) - 1e-3, softcap + np.log(700) + 1e-3
     assert np.all(got["lse"] >= lo) and np.all(got["lse"] <= hi)
     assert_parity(got, ref)
+
+
+def test_forward_backward_replay_in_a_cuda_graph(dev):
+    """After one eager call (which does the per-device set-up), forward + backward
+    only enqueue kernels on the caller's stream, so the pair can be captured
+    into a CUDA graph and replayed; replays match the eager results bit for bit."""
+    w = CASES["ktail_softcap_padded"]
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    n, h = hid.shape
+    ws = torch.empty(flce.workspace_size(n, h, wt.shape[0], w.vocab), dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, device=dev)
+    lse = torch.empty(n, device=dev)
+    dh = torch.empty_like(hid)
+    dw = torch.empty_like(wt)
+    grad = torch.ones(1, device=dev)
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab, workspace=ws)
+
+    def step():
+        flce.forward(hid, wt, lab, loss=loss, lse=lse, **kw)
+        flce.backward(hid, wt, lab, lse, grad, dhidden=dh, dweight=dw, **kw)
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        step()                                   # eager warm-up on the capture stream
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    eager = [t.clone() for t in (loss, lse, dh, dw)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for _ in range(3):
+        for t in (loss, lse, dh, dw):
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for a, b in zip(eager, (loss, lse, dh, dw)):
+            assert torch.equal(a, b)
+    assert flce.get_error(dev) == flce.FLCE_OK
