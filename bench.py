@@ -369,7 +369,10 @@ def run_ours(args, w) -> int:
 
     ms, launches, stats, clocks = timed_region()
     remeasured = False
-    if BAD_REASONS & set(clocks.get("reasons", [])):
+    # Re-measure once if any rank saw a hardware or thermal slowdown; the
+    # decision is collective so every rank takes the same barriers.
+    bad = 1.0 if BAD_REASONS & set(clocks.get("reasons", [])) else 0.0
+    if max_over_ranks(bad) > 0:
         ms, launches, stats, clocks = timed_region()
         remeasured = True
     ms_max = max_over_ranks(ms)
@@ -411,8 +414,11 @@ def run_ours(args, w) -> int:
     dom_name = max(gemms, key=lambda k: gemms[k]["total_ms"])
     dom = gemms[dom_name]
     achieved = dom["flops"] / (dom["total_ms"] / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    # The kernels are timed inside a seconds-long continuous run (clocks settle
+    # under the power cap), so the sustained GEMM figure is the denominator;
+    # the burst figure is reported beside it.
+    peak_burst = float(peaks["bf16_tflops"])
+    peak = float(peaks.get("bf16_tflops_sustained", peak_burst))
     per_step_launches = dom["launches"] / args.steps
     traffic = committed_traffic(w.name, dom_name)
     kernels = {k: {"launches_per_step": s["launches"] / args.steps,
@@ -434,10 +440,11 @@ def run_ours(args, w) -> int:
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + write.sum)",
                 "flops_per_launch": dom["flops"] / dom["launches"],
                 "launches_per_step": per_step_launches,
-                "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "peak_sustained": peak_sus, "frac_of_sustained": achieved / peak_sus,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS, seconds-long loop)",
+                "peak_burst": peak_burst, "frac_of_burst": achieved / peak_burst,
                 "whole_path_tflops": path_flops / (ms_max / 1e3) / 1e12 / world,
                 "whole_path_frac": path_flops / (ms_max / 1e3) / 1e12 / world / peak,
+                "whole_path_frac_of_burst": path_flops / (ms_max / 1e3) / 1e12 / world / peak_burst,
             },
             "kernels": kernels,
             "e2e": {"value": e2e_value, "unit": UNIT,
