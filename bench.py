@@ -313,6 +313,8 @@ def run_ours(args, w) -> int:
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, dev)
 
+    from lm_head_projection_flce_b200 import build as B
+    B.build()                               # no-op when the in-tree library matches its sources
     flce.load_library()
     d = W.generate(w)                       # seeded on the CPU: the same batch on every rank
     hid = d["hidden"].to(dev)
@@ -474,6 +476,8 @@ def run_chunked_ce(args) -> int:
         raise RuntimeError("bench.py needs a CUDA device (sm_100a)")
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
+    from lm_head_projection_flce_b200 import build as B
+    B.build()
     flce.load_library()
     w = W.CE_LOGITS
     d = W.generate_logits(w)

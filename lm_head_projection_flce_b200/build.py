@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import argparse
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -20,6 +21,7 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libflce.so")
+DIGEST_PATH = LIB_PATH + ".sources"  # sha256 of the sources the library was built from
 MAIN_SOURCE = os.path.join(CSRC, "flce.cu")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -39,19 +41,31 @@ def sources() -> list[str]:
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in sources():
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    h.update(" ".join(ARCH_FLAGS + NVCC_FLAGS).encode())
+    return h.hexdigest()
+
+
 def is_stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+    """True when the library is missing or was built from other sources or flags
+    (compared by content, so copying the tree does not force a rebuild)."""
+    if not os.path.exists(LIB_PATH) or not os.path.exists(DIGEST_PATH):
         return True
-    t = os.path.getmtime(LIB_PATH)
-    return any(os.path.getmtime(s) > t for s in sources())
+    with open(DIGEST_PATH) as f:
+        return f.read().strip() != source_digest()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile libflce.so if missing or older than its sources; return its path."""
     if not force and not is_stale():
         return LIB_PATH
-    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", "-o", LIB_PATH + ".tmp",
-           MAIN_SOURCE]
+    tmp = f"{LIB_PATH}.tmp{os.getpid()}"  # concurrent builders never share a temp file
+    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", "-o", tmp, MAIN_SOURCE]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -60,7 +74,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr, flush=True)
-    os.replace(LIB_PATH + ".tmp", LIB_PATH)
+    digest = source_digest()
+    os.replace(tmp, LIB_PATH)
+    with open(f"{DIGEST_PATH}.tmp{os.getpid()}", "w") as f:
+        f.write(digest + "\n")
+    os.replace(f"{DIGEST_PATH}.tmp{os.getpid()}", DIGEST_PATH)
     return LIB_PATH
 
 
