@@ -22,6 +22,10 @@
 //   K3(c+1)} whose CTAs take tiles dynamically, long K5 tiles first, so no
 //   launch ends on a partial wave of long tiles
 //   zero    dW rows [V, Vp)
+// Every GEMM above runs on the CTA-pair kernel of gemm_sm100_pair.cuh (256 x
+// 256 tiles, tcgen05 cta_group::2); the epilogues are in epilogues.cuh.
+// Cross entropy on given logits (chunked_ce page) is at the end of this file,
+// its row kernels in chunked_ce.cuh; the forward without allocation at the end.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
