@@ -92,11 +92,14 @@ __global__ void zero16_kernel(uint4* __restrict__ dst, int64_t n16) {
 }
 
 // K2: merge the per-tile partials of 32 token rows (8 warps split the tiles),
-// then per token: lse, token loss, label check; per block: loss and count sums.
+// then per token: lse, token loss, label check (mask: optional, 0 = ignore the
+// token); per block: loss and count sums.  Also finishes the cross entropy on
+// given logits, whose row segments leave partials in the same layout.
 __global__ void __launch_bounds__(kMergeRows* kMergeWarps)
     lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
                      int v_tiles, int64_t n_tokens, const float* __restrict__ label_logit,
-                     const int64_t* __restrict__ labels, int64_t vocab, int64_t ignore_index,
+                     const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
+                     int64_t vocab, int64_t ignore_index,
                      float* __restrict__ lse_out, float* __restrict__ token_loss,
                      double* __restrict__ blk_loss, int* __restrict__ blk_cnt,
                      unsigned* __restrict__ err) {
@@ -109,6 +112,7 @@ __global__ void __launch_bounds__(kMergeRows* kMergeWarps)
     for (int t = warp; t < v_tiles; t += kMergeWarps) {
       const float m = part_m[int64_t(t) * n_tokens + n];
       const float s = part_s[int64_t(t) * n_tokens + n];
+      if (m == -INFINITY) continue;  // an empty partial (or one of only -inf logits)
       const float mn = fmaxf(M, m);
       S = S * exp2f(M - mn) + s * exp2f(m - mn);
       M = mn;
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(kMergeRows* kMergeWarps)
   if (n < n_tokens) {
     const float lse = (Mt + log2f(St)) * 0.6931471805599453f;
     const int64_t y = labels[n];
-    bool valid = y != ignore_index;
+    bool valid = y != ignore_index && (mask == nullptr || mask[n] != 0);
     if (valid && (y < 0 || y >= vocab)) {
       atomicOr(err, kDevErrBadLabel);
       valid = false;
@@ -258,6 +262,7 @@ struct DeviceInfo {
   int status = FLCE_OK;
   int num_sms = 0;
   int max_pairs = 0;  // CTA pairs of the pair GEMM that fit at once (0 = not yet queried)
+  int ce_blocks[4] = {};  // resident CTAs per SM of the CE kernels (0 = not yet queried)
   unsigned* err = nullptr;
 };
 
@@ -723,8 +728,8 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   {
     LaunchScope scope(KF_MERGE, 0.0, 8.0 * double(p.v_tiles) * n + 24.0 * n, cs);
     lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
-        ep.part_m, ep.part_s, int(p.v_tiles), n, ep.label_logit, labels, v, ignore_index, lse,
-        reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
+        ep.part_m, ep.part_s, int(p.v_tiles), n, ep.label_logit, labels, nullptr, v,
+        ignore_index, lse, reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
   }
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   if (reduction != FLCE_NONE) {
@@ -1085,14 +1090,22 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
 namespace flce {
 
 struct CePlan {
-  size_t off_loss, off_cnt, off_lse2, off_scale, total;
+  size_t off_pm, off_ps, off_zl, off_bl, off_bc, off_lse2, off_scale, total;
+  int64_t nblk;
 };
 
+// Workspace: per-segment partials for up to kCeMaxSplits segments per row,
+// the label logits, the merge blocks' loss sums and the backward's per-token
+// lse * log2 e and gradient scale.
 static CePlan plan_ce(int64_t n) {
   CePlan p{};
+  p.nblk = cdiv(n, kMergeRows);
   size_t o = 0;
-  p.off_loss = o;  o = align_up(o + size_t(n) * 8);
-  p.off_cnt = o;   o = align_up(o + size_t(n) * 4);
+  p.off_pm = o;    o = align_up(o + size_t(n) * kCeMaxSplits * 4);
+  p.off_ps = o;    o = align_up(o + size_t(n) * kCeMaxSplits * 4);
+  p.off_zl = o;    o = align_up(o + size_t(n) * 4);
+  p.off_bl = o;    o = align_up(o + size_t(p.nblk) * 8);
+  p.off_bc = o;    o = align_up(o + size_t(p.nblk) * 4);
   p.off_lse2 = o;  o = align_up(o + size_t(n) * 4);
   p.off_scale = o; o = align_up(o + size_t(n) * 4);
   p.total = std::max(o, kAlign);
@@ -1114,8 +1127,39 @@ static int check_ce(const void* logits, int dtype, const int64_t* labels, int64_
   return FLCE_OK;
 }
 
-static int ce_grid(const DeviceInfo& dev, int64_t n) {
-  return int(std::min<int64_t>(n, int64_t(dev.num_sms) * 16));
+// Launch shape of a CE kernel: whole rows per CTA (grid-stride, up to 16
+// CTAs per SM, the hardware scheduler fills slots as CTAs finish).  When the
+// rows are fewer than the resident CTA slots (queried once per device and
+// kernel), rows are cut into segments of at least kCeMinSegment elements so
+// every slot gets work; longer units keep each CTA's load pipeline full.
+struct CeLaunch {
+  int grid, splits;
+};
+
+template <typename Kernel>
+static CeLaunch ce_launch(DeviceInfo& dev, int which, Kernel kern, int smem, int64_t n,
+                          int64_t v) {
+  int per_sm = dev.ce_blocks[which];
+  if (per_sm == 0) {  // first launch of this kernel on this device
+    if (smem > 0 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+      return CeLaunch{0, 0};
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCeThreads, smem) !=
+            cudaSuccess ||
+        per_sm <= 0)
+      per_sm = 1;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    dev.ce_blocks[which] = per_sm;
+  }
+  const int64_t slots = int64_t(per_sm) * dev.num_sms;
+  CeLaunch l;
+  l.splits = 1;
+  if (n < slots)
+    l.splits = int(std::max<int64_t>(
+        1, std::min<int64_t>({kCeMaxSplits, slots / std::max<int64_t>(n, 1), v / kCeMinSegment})));
+  l.grid = int(std::min<int64_t>(n * l.splits, int64_t(dev.num_sms) * 16));
+  return l;
 }
 
 }  // namespace flce
@@ -1142,25 +1186,42 @@ extern "C" int flce_ce_forward(const void* logits, int dtype, const int64_t* lab
   if ((st = device_info(&dev)) != FLCE_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  double* row_loss = reinterpret_cast<double*>(ws + p.off_loss);
-  int* row_cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  float* part_m = reinterpret_cast<float*>(ws + p.off_pm);
+  float* part_s = reinterpret_cast<float*>(ws + p.off_ps);
+  float* label_logit = reinterpret_cast<float*>(ws + p.off_zl);
+  double* blk_loss = reinterpret_cast<double*>(ws + p.off_bl);
+  int* blk_cnt = reinterpret_cast<int*>(ws + p.off_bc);
   if (n > 0) {
     const size_t esz = dtype == FLCE_F32 ? 4 : 2;
-    LaunchScope scope(KF_CE_FWD, 0.0, double(n) * double(v) * esz + 24.0 * double(n), cs);
-    float* tok = reduction == FLCE_NONE ? loss : nullptr;
-    if (dtype == FLCE_BF16)
-      ce_forward_kernel<__nv_bfloat16><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
-          static_cast<const __nv_bfloat16*>(logits), ld, labels, mask, n, v, ignore_index, lse,
-          tok, row_loss, row_cnt, dev->err);
-    else
-      ce_forward_kernel<float><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
-          static_cast<const float*>(logits), ld, labels, mask, n, v, ignore_index, lse, tok,
-          row_loss, row_cnt, dev->err);
+    CeLaunch l;
+    {
+      LaunchScope scope(KF_CE_FWD, 0.0, double(n) * double(v) * esz + 24.0 * double(n), cs);
+      if (dtype == FLCE_BF16) {
+        auto kern = ce_partials_kernel<__nv_bfloat16>;
+        l = ce_launch(*dev, 0, kern, 0, n, v);
+        if (l.grid == 0) return FLCE_ERR_CUDA;
+        kern<<<l.grid, kCeThreads, 0, cs>>>(
+            static_cast<const __nv_bfloat16*>(logits), ld, labels, mask, n, v, ignore_index,
+            l.splits, part_m, part_s, label_logit);
+      } else {
+        auto kern = ce_partials_kernel<float>;
+        l = ce_launch(*dev, 1, kern, 0, n, v);
+        if (l.grid == 0) return FLCE_ERR_CUDA;
+        kern<<<l.grid, kCeThreads, 0, cs>>>(
+            static_cast<const float*>(logits), ld, labels, mask, n, v, ignore_index, l.splits,
+            part_m, part_s, label_logit);
+      }
+    }
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    LaunchScope scope(KF_MERGE, 0.0, 8.0 * double(l.splits) * double(n) + 24.0 * double(n), cs);
+    lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
+        part_m, part_s, l.splits, n, label_logit, labels, mask, v, ignore_index, lse,
+        reduction == FLCE_NONE ? loss : nullptr, blk_loss, blk_cnt, dev->err);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
   if (reduction != FLCE_NONE) {
-    LaunchScope scope(KF_FINAL, 0.0, 12.0 * double(n), cs);
-    loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(row_loss, row_cnt, int(n), reduction,
+    LaunchScope scope(KF_FINAL, 0.0, 12.0 * double(p.nblk), cs);
+    loss_finalize_kernel<<<1, kFinalThreads, 0, cs>>>(blk_loss, blk_cnt, int(p.nblk), reduction,
                                                       num_label_tokens, loss);
     if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   }
@@ -1198,13 +1259,20 @@ extern "C" int flce_ce_backward(const void* logits, int dtype, const int64_t* la
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   const size_t esz = dtype == FLCE_F32 ? 4 : 2;
   LaunchScope scope(KF_CE_BWD, 0.0, 2.0 * double(n) * double(v) * esz + 16.0 * double(n), cs);
-  if (dtype == FLCE_BF16)
-    ce_backward_kernel<__nv_bfloat16><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
-        static_cast<const __nv_bfloat16*>(logits), ld, labels, n, v, lse2, scale,
+  if (dtype == FLCE_BF16) {
+    auto kern = ce_backward_kernel<__nv_bfloat16>;
+    const CeLaunch l = ce_launch(*dev, 2, kern, kCeRingBytes, n, v);
+    if (l.grid == 0) return FLCE_ERR_CUDA;
+    kern<<<l.grid, kCeThreads, kCeRingBytes, cs>>>(
+        static_cast<const __nv_bfloat16*>(logits), ld, labels, n, v, l.splits, lse2, scale,
         static_cast<__nv_bfloat16*>(dlogits));
-  else
-    ce_backward_kernel<float><<<ce_grid(*dev, n), kCeThreads, 0, cs>>>(
-        static_cast<const float*>(logits), ld, labels, n, v, lse2, scale,
-        static_cast<float*>(dlogits));
+  } else {
+    auto kern = ce_backward_kernel<float>;
+    const CeLaunch l = ce_launch(*dev, 3, kern, kCeRingBytes, n, v);
+    if (l.grid == 0) return FLCE_ERR_CUDA;
+    kern<<<l.grid, kCeThreads, kCeRingBytes, cs>>>(static_cast<const float*>(logits), ld, labels,
+                                                   n, v, l.splits, lse2, scale,
+                                                   static_cast<float*>(dlogits));
+  }
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }

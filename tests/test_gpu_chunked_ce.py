@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from lm_head_projection_flce_b200 import flce
+from lm_head_projection_flce_b200 import workloads as W
 from oracle import flce_oracle as O
 
 from gpu_common import GRAD_REL, LOSS_REL, LSE_ABS, gpu_device, max_rel
@@ -136,3 +137,71 @@ def test_ce_matches_fused_path_on_materialised_logits(dev):
     torch.cuda.synchronize(dev)
     assert torch.allclose(lse1, lse2, atol=1e-3, rtol=0)
     assert abs(float(l1) - float(l2)) <= 1e-4 * abs(float(l2))
+
+
+@pytest.mark.parametrize("dtype,ld", [(torch.bfloat16, 20013), (torch.float32, 20011)])
+def test_ce_multi_segment_rows_unaligned_with_mask(dev, dtype, ld):
+    """Rows long enough to be cut into several segments, each row starting at
+    a different 16-byte phase, with a mask and a row stride."""
+    n, v = 70, 20009
+    full, logits, labels = _case(11, n, v, dtype, ld=ld)
+    mask = (torch.arange(n) % 7 != 3).to(torch.uint8)
+    z = full.to(dev)[:, :v]
+    lab = labels.to(dev)
+    loss, lse = flce.ce_forward(z, lab, mask=mask.to(dev))
+    dbuf = torch.full((n, ld), 7.0, dtype=dtype, device=dev)
+    flce.ce_backward(z, lab, lse, torch.ones(1, device=dev), mask=mask.to(dev),
+                     dlogits=dbuf[:, :v])
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
+    zf = logits.double().numpy()
+    ref = O.ce_forward(zf, labels.numpy(), mask=mask.numpy())
+    rdz = O.ce_backward(zf, labels.numpy(), mask=mask.numpy())
+    assert float(np.max(np.abs(lse.double().cpu().numpy() - ref.lse))) <= LSE_ABS
+    assert abs(float(loss) - ref.loss) <= LOSS_REL * abs(ref.loss)
+    assert max_rel(dbuf[:, :v].double().cpu().numpy(), rdz) <= GRAD_REL
+    assert torch.all(dbuf[:, v:] == 7.0)
+    assert torch.all(dbuf[3::7, :v] == 0)
+
+
+def test_ce_segments_of_only_minus_infinity(dev):
+    """A row whose leading segments hold only -inf logits (masked vocabulary
+    entries): their partials are empty and must not poison the merge."""
+    n, v = 40, 20000
+    _, logits, labels = _case(12, n, v, torch.bfloat16, ignore_frac=0.0)
+    logits[:10, :12000] = float("-inf")
+    labels[:10] = torch.randint(12000, v, (10,), generator=torch.Generator().manual_seed(3))
+    dz = _check(dev, logits, labels)
+    assert torch.all(dz[:10, :12000] == 0)
+
+
+def test_ce_full_size_bench_workload(dev):
+    """The benchmark's logits [4096, 128256] BF16 in the launch configuration
+    bench.py times: lse and the loss for every row, dlogits on sampled rows."""
+    w = W.CE_LOGITS
+    d = W.generate_logits(w)
+    logits, labels, nlt = d["logits"], d["labels"], d["num_label_tokens"]
+    z = logits.to(dev)
+    lab = labels.to(dev)
+    loss, lse = flce.ce_forward(z, lab, reduction=w.reduction, num_label_tokens=nlt)
+    dz = flce.ce_backward(z, lab, lse, torch.ones(1, device=dev), reduction=w.reduction,
+                          num_label_tokens=nlt)
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
+    lse_g = lse.double().cpu().numpy()
+    tok = np.zeros(w.n_tokens)
+    worst = 0.0
+    for r0 in range(0, w.n_tokens, 512):
+        blk = logits[r0:r0 + 512].double().numpy()
+        ref = O.ce_forward(blk, labels[r0:r0 + 512].numpy(), reduction="none")
+        worst = max(worst, float(np.max(np.abs(lse_g[r0:r0 + 512] - ref.lse))))
+        tok[r0:r0 + 512] = ref.loss
+    assert worst <= LSE_ABS
+    ref_total = float(tok.sum()) / nlt
+    assert abs(float(loss) - ref_total) <= LOSS_REL * abs(ref_total)
+    rows = torch.randperm(w.n_tokens, generator=torch.Generator().manual_seed(5))[:48]
+    ignored = torch.nonzero(labels == II)[:4, 0]
+    rows = torch.cat([rows, ignored, torch.tensor([0, w.n_tokens - 1])]).unique()
+    sub = logits[rows].double().numpy()
+    rdz = O.ce_backward(sub, labels[rows].numpy(), reduction=w.reduction, num_label_tokens=nlt)
+    assert max_rel(dz[rows.to(dev)].double().cpu().numpy(), rdz) <= GRAD_REL
