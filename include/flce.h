@@ -32,10 +32,11 @@
  *    aborts across this boundary.  FLCE_ERR_CUDA from a launch means kernels
  *    the call enqueued before it may still run; the call's outputs are then
  *    undefined.
- *  - After one call per device (which queries the device and resolves the
- *    tensor-map encoder), flce_forward / flce_backward / flce_ce_* only
- *    enqueue kernels on `stream`, so a sequence of them can be captured into
- *    a CUDA graph and replayed with the same buffers.
+ *  - After one call of an entry point per device and dtype (which queries the
+ *    device, resolves the tensor-map encoder and caches launch shapes),
+ *    flce_forward / flce_backward / flce_ce_* only enqueue kernels on
+ *    `stream`, so a sequence of them can be captured into a CUDA graph and
+ *    replayed with the same buffers.
  *  - Labels outside [0, V) that are not ignore_index cannot be checked on the
  *    host without a device read; the kernels treat them as ignored (zero loss,
  *    zero gradient) and raise FLCE_ERR_BAD_LABEL in a per-device error word

@@ -147,10 +147,31 @@ def _prepare(hidden, weight, labels):
     return hid, lab
 
 
-def _workspace(ws, need: int, device) -> torch.Tensor:
+def _workspace(ws, need: int, device) -> tuple[torch.Tensor, int]:
+    """The workspace tensor and its size in bytes (any dtype; contiguous, on `device`)."""
     if ws is None:
-        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
-    return ws
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    elif ws.device != device or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the inputs' device")
+    return ws, ws.numel() * ws.element_size()
+
+
+def _buffer(t, numel: int, dtype, device, name: str) -> torch.Tensor:
+    """A caller-supplied buffer the library reads or writes through a raw pointer:
+    it must have exactly the expected dtype, size and device, and be contiguous."""
+    if t.dtype != dtype or t.numel() != numel or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of {numel} elements on "
+                         f"{device}")
+    return t
+
+
+def _forward_outputs(loss, lse, n: int, reduction: str, dev):
+    loss_n = n if reduction == "none" else 1
+    loss = (torch.empty(loss_n, dtype=torch.float32, device=dev) if loss is None
+            else _buffer(loss, loss_n, torch.float32, dev, "loss"))
+    lse = (torch.empty(n, dtype=torch.float32, device=dev) if lse is None
+           else _buffer(lse, n, torch.float32, dev, "lse"))
+    return loss, lse
 
 
 def forward(hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
@@ -165,16 +186,22 @@ def forward(hidden, weight, labels, *, ignore_index: int = -100, softcap: float 
     v = _vocab(weight, unpadded_vocab)
     dev = hid.device
     red = REDUCTIONS[reduction]
-    if loss is None:
-        loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
-    if lse is None:
-        lse = torch.empty(n, dtype=torch.float32, device=dev)
-    ws = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
+    loss, lse = _forward_outputs(loss, lse, n, reduction, dev)
+    ws, ws_bytes = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
     st = lib.flce_forward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
                           v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
-                          _ptr(loss), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(dev, stream))
+                          _ptr(loss), _ptr(lse), _ptr(ws), ws_bytes, _stream_handle(dev, stream))
     _check("flce_forward", st)
     return (loss if reduction == "none" else loss.reshape(())), lse
+
+
+def _grad_loss(grad_loss, n: int, reduction: str, dev) -> torch.Tensor:
+    """The upstream gradient as FP32 on the device: [N] for 'none', else one value."""
+    grad = torch.as_tensor(grad_loss).reshape(-1).to(device=dev, dtype=torch.float32).contiguous()
+    if grad.numel() != (n if reduction == "none" else 1):
+        raise ValueError("grad_loss must have one value per token for reduction='none', "
+                         "else one value")
+    return grad
 
 
 def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100,
@@ -190,16 +217,17 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
     v = _vocab(weight, unpadded_vocab)
     dev = hid.device
     red = REDUCTIONS[reduction]
-    grad = grad_loss.reshape(-1).to(device=dev, dtype=torch.float32).contiguous()
-    if dhidden is None:
-        dhidden = torch.empty_like(hid)
-    if dweight is None:
-        dweight = torch.empty_like(weight)
-    ws = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
+    grad = _grad_loss(grad_loss, n, reduction, dev)
+    lse = _buffer(lse, n, torch.float32, dev, "lse")
+    dhidden = (torch.empty_like(hid) if dhidden is None
+               else _buffer(dhidden, n * h, torch.bfloat16, dev, "dhidden"))
+    dweight = (torch.empty_like(weight) if dweight is None
+               else _buffer(dweight, weight.numel(), weight.dtype, dev, "dweight"))
+    ws, ws_bytes = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
     st = lib.flce_backward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
                            v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
                            _ptr(grad), _ptr(lse), _ptr(dhidden), _ptr(dweight), _ptr(ws),
-                           ws.numel(), _stream_handle(dev, stream))
+                           ws_bytes, _stream_handle(dev, stream))
     _check("flce_backward", st)
     return dhidden.reshape(hidden.shape), dweight
 
@@ -296,10 +324,7 @@ def forward_noalloc(hidden, weight, labels, *, ignore_index: int = -100, softcap
     vp = weight.shape[0]
     v = _vocab(weight, unpadded_vocab)
     dev = hid.device
-    if loss is None:
-        loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
-    if lse is None:
-        lse = torch.empty(n, dtype=torch.float32, device=dev)
+    loss, lse = _forward_outputs(loss, lse, n, reduction, dev)
     st = lib.flce_forward_noalloc(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n,
                                   h, vp, v, ignore_index, float(softcap), REDUCTIONS[reduction],
                                   int(num_label_tokens or 0), _ptr(loss), _ptr(lse),
@@ -334,18 +359,18 @@ def _prepare_logits(logits, labels, mask):
 
 
 def ce_forward(logits, labels, *, mask=None, ignore_index: int = -100, reduction: str = "sum",
-               num_label_tokens: int | None = None, workspace=None, stream=None):
+               num_label_tokens: int | None = None, workspace=None,
+               loss: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
     """Cross entropy of given logits [..., V] (ChunkedCrossEntropy).  Returns (loss, lse)."""
     lib = load_library()
     z, lab, m = _prepare_logits(logits, labels, mask)
     n, v = z.shape
     dev = z.device
-    loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
-    lse = torch.empty(n, dtype=torch.float32, device=dev)
-    ws = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
+    loss, lse = _forward_outputs(loss, lse, n, reduction, dev)
+    ws, ws_bytes = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
     st = lib.flce_ce_forward(_ptr(z), W_DTYPES[z.dtype], _ptr(lab), _ptr(m), n, v, z.stride(0),
                              ignore_index, REDUCTIONS[reduction], int(num_label_tokens or 0),
-                             _ptr(loss), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(dev, stream))
+                             _ptr(loss), _ptr(lse), _ptr(ws), ws_bytes, _stream_handle(dev, stream))
     _check("flce_ce_forward", st)
     return (loss if reduction == "none" else loss.reshape(())), lse
 
@@ -358,16 +383,19 @@ def ce_backward(logits, labels, lse, grad_loss, *, mask=None, ignore_index: int 
     z, lab, m = _prepare_logits(logits, labels, mask)
     n, v = z.shape
     dev = z.device
-    grad = grad_loss.reshape(-1).to(device=dev, dtype=torch.float32).contiguous()
+    grad = _grad_loss(grad_loss, n, reduction, dev)
+    lse = _buffer(lse, n, torch.float32, dev, "lse")
     if dlogits is None:
         dlogits = torch.empty_like(z)
     out = dlogits.reshape(n, v)
+    if out.dtype != z.dtype or out.device != dev:
+        raise ValueError("dlogits must have the logits' dtype and device")
     if out.stride(0) != z.stride(0) or out.stride(1) != 1:
         raise ValueError("dlogits must have the logits' row stride")
-    ws = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
+    ws, ws_bytes = _workspace(workspace, int(lib.flce_ce_workspace_size(n)), dev)
     st = lib.flce_ce_backward(_ptr(z), W_DTYPES[z.dtype], _ptr(lab), _ptr(m), n, v, z.stride(0),
                               ignore_index, REDUCTIONS[reduction], int(num_label_tokens or 0),
-                              _ptr(grad), _ptr(lse), _ptr(out), _ptr(ws), ws.numel(),
+                              _ptr(grad), _ptr(lse), _ptr(out), _ptr(ws), ws_bytes,
                               _stream_handle(dev, stream))
     _check("flce_ce_backward", st)
     return out.reshape(logits.shape)

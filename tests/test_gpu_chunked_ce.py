@@ -205,3 +205,41 @@ def test_ce_full_size_bench_workload(dev):
     sub = logits[rows].double().numpy()
     rdz = O.ce_backward(sub, labels[rows].numpy(), reduction=w.reduction, num_label_tokens=nlt)
     assert max_rel(dz[rows.to(dev)].double().cpu().numpy(), rdz) <= GRAD_REL
+
+
+@pytest.mark.parametrize("n,v", [(300, 50001), (40, 70000)])
+def test_ce_replay_in_a_cuda_graph(dev, n, v):
+    """After one eager call (per-device set-up and launch shapes), forward +
+    backward only enqueue kernels, so they can be captured into a CUDA graph
+    and replayed bit for bit; the second shape cuts its rows into segments."""
+    _, logits, labels = _case(13, n, v, torch.bfloat16)
+    z, lab = logits.to(dev), labels.to(dev)
+    ws = torch.empty(int(flce.load_library().flce_ce_workspace_size(n)), dtype=torch.uint8,
+                     device=dev)
+    loss = torch.empty(1, device=dev)
+    lse = torch.empty(n, device=dev)
+    dz = torch.empty_like(z)
+    grad = torch.ones(1, device=dev)
+
+    def step():
+        flce.ce_forward(z, lab, loss=loss, lse=lse, workspace=ws)
+        flce.ce_backward(z, lab, lse, grad, dlogits=dz, workspace=ws)
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    eager = [t.clone() for t in (loss, lse, dz)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for _ in range(2):
+        for t in (loss, lse, dz):
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for a, b in zip(eager, (loss, lse, dz)):
+            assert torch.equal(a, b)
+    assert flce.get_error(dev) == flce.FLCE_OK

@@ -293,3 +293,37 @@ def test_forward_backward_replay_in_a_cuda_graph(dev):
         for a, b in zip(eager, (loss, lse, dh, dw)):
             assert torch.equal(a, b)
     assert flce.get_error(dev) == flce.FLCE_OK
+
+
+def test_binding_refuses_mismatched_buffers(dev):
+    """Caller-supplied outputs, lse and workspace reach the library as raw
+    pointers, so the binding refuses any of the wrong dtype, size or layout
+    before a kernel could write past them."""
+    w = CASES["ktail_softcap_padded"]
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    n, h = hid.reshape(-1, hid.shape[-1]).shape
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab)
+    loss, lse = flce.forward(hid, wt, lab, **kw)
+    g = torch.ones(1, device=dev)
+    bad = [
+        lambda: flce.forward(hid, wt, lab, lse=torch.empty(n - 1, device=dev), **kw),
+        lambda: flce.forward(hid, wt, lab, loss=torch.empty(2, device=dev), **kw),
+        lambda: flce.forward(hid, wt, lab, lse=torch.empty(n, device=dev, dtype=torch.float64),
+                             **kw),
+        lambda: flce.backward(hid, wt, lab, lse[:-1], g, **kw),
+        lambda: flce.backward(hid, wt, lab, lse, torch.ones(2, device=dev), **kw),
+        lambda: flce.backward(hid, wt, lab, lse, g, **kw,
+                              dhidden=torch.empty(n, h - 8, device=dev, dtype=torch.bfloat16)),
+        lambda: flce.backward(hid, wt, lab, lse, g, **kw,
+                              dweight=torch.empty_like(wt, dtype=torch.float16)),
+        lambda: flce.backward(hid, wt, lab, lse, g, **kw,
+                              dweight=torch.empty(wt.shape[1], wt.shape[0], device=dev,
+                                                  dtype=wt.dtype).t()),
+        lambda: flce.forward(hid, wt, lab, workspace=torch.empty(64, 64, device=dev).t(), **kw),
+    ]
+    for call in bad:
+        with pytest.raises(ValueError):
+            call()
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
