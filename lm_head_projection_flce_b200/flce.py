@@ -386,7 +386,8 @@ def ce_backward(logits, labels, lse, grad_loss, *, mask=None, ignore_index: int 
     grad = _grad_loss(grad_loss, n, reduction, dev)
     lse = _buffer(lse, n, torch.float32, dev, "lse")
     if dlogits is None:
-        dlogits = torch.empty_like(z)
+        # the kernels write dlogits with the logits' row stride
+        dlogits = torch.empty(n, z.stride(0), dtype=z.dtype, device=dev)[:, :v]
     out = dlogits.reshape(n, v)
     if out.dtype != z.dtype or out.device != dev:
         raise ValueError("dlogits must have the logits' dtype and device")

@@ -327,3 +327,54 @@ def test_binding_refuses_mismatched_buffers(dev):
             call()
     torch.cuda.synchronize(dev)
     assert flce.get_error(dev) == flce.FLCE_OK
+
+
+def test_fp32_head_chunkings_noalloc_and_graph_replay(dev):
+    """FP32 head (cast to BF16 inside each call): the same results for every
+    backward chunking, flce_forward_noalloc equals flce_forward bit for bit,
+    and a captured forward + backward replays bit for bit."""
+    w = W.custom(300, 264, 5000, 5120, w_dtype="f32", softcap=30.0, ignore_frac=0.1, seed=21)
+    d = W.generate(w)
+    ref = run_oracle(d, w)
+    lo = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, torch.float32,
+                             minimum=True)
+    hi = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, torch.float32)
+    for ws in (lo, lo + 2 * w.n_tokens * 256 * 4, hi):   # 20, 7 and 5 backward chunks
+        assert_parity(run_gpu(d, w, dev, ws_bytes=ws), ref)
+
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab)
+    loss_a, lse_a = flce.forward(hid, wt, lab, **kw)
+    loss_b, lse_b = flce.forward_noalloc(hid, wt, lab, **kw)
+    torch.cuda.synchronize(dev)
+    assert torch.equal(loss_a, loss_b) and torch.equal(lse_a, lse_b)
+
+    ws = torch.empty(lo + 2 * w.n_tokens * 256 * 4, dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, device=dev)
+    lse = torch.empty(w.n_tokens, device=dev)
+    dh = torch.empty_like(hid)
+    dw = torch.empty_like(wt)
+    grad = torch.ones(1, device=dev)
+
+    def step():
+        flce.forward(hid, wt, lab, loss=loss, lse=lse, workspace=ws, **kw)
+        flce.backward(hid, wt, lab, lse, grad, dhidden=dh, dweight=dw, workspace=ws, **kw)
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    eager = [t.clone() for t in (loss, lse, dh, dw)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for _ in range(2):
+        for t in (loss, lse, dh, dw):
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for a, b in zip(eager, (loss, lse, dh, dw)):
+            assert torch.equal(a, b)
+    assert flce.get_error(dev) == flce.FLCE_OK

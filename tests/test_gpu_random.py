@@ -71,3 +71,53 @@ def test_random_case(dev, i):
     rdh, rdw = O.backward(d["hidden"].double().numpy(), hw, labels.numpy(),
                           grad_loss=grad.double().numpy(), **kw)
     assert_parity(got, {"loss": np.asarray(fwd.loss), "lse": fwd.lse, "dh": rdh, "dw": rdw}), c
+
+
+def _draw_ce(i):
+    r = np.random.default_rng(900 + i)
+    n = int(r.choice([int(r.integers(1, 64)), int(r.integers(64, 600)), int(r.integers(600, 1500))]))
+    v = int(r.choice([int(r.integers(1, 3000)), int(r.integers(30000, 140000))]))
+    v = max(1, min(v, 40_000_000 // n))        # keep the FP64 oracle to a few seconds
+    return dict(n=n, v=v, pad=int(r.choice([0, 0, 1, 3, 17])),
+                dtype=str(r.choice(["bf16", "f32"])),
+                scale=float(r.choice([1.0, 3.0, 8.0])),
+                reduction=str(r.choice(["sum", "sum", "mean", "none"])),
+                norm=bool(r.integers(0, 2)), mask=bool(r.integers(0, 2)),
+                ignore_frac=float(r.choice([0.0, 0.1, 0.5])), seed=950 + i)
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_random_ce_case(dev, i):
+    """Cross entropy on given logits: row counts below and above the resident
+    CTA slots (segmented and whole-row launches), long and short rows, row
+    strides, masks, both dtypes, every reduction, against the FP64 oracle."""
+    c = _draw_ce(i)
+    g = torch.Generator().manual_seed(c["seed"])
+    n, v, ld = c["n"], c["v"], c["v"] + c["pad"]
+    dtype = torch.float32 if c["dtype"] == "f32" else torch.bfloat16
+    full = (torch.randn(n, ld, generator=g) * c["scale"]).to(dtype)
+    labels = torch.randint(0, v, (n,), generator=g)
+    k = int(c["ignore_frac"] * n + 0.5)
+    if k:
+        labels[torch.randperm(n, generator=g)[:k]] = W.IGNORE_INDEX
+    mask = (torch.rand(n, generator=g) > 0.2).to(torch.uint8) if c["mask"] else None
+    red = c["reduction"]
+    valid = (labels != W.IGNORE_INDEX) & (mask.bool() if mask is not None else True)
+    nvalid = int(valid.sum())
+    nlt = nvalid if (red == "sum" and c["norm"] and nvalid > 0) else None
+    z = full.to(dev)[:, :v]
+    m = mask.to(dev) if mask is not None else None
+    grad = torch.linspace(-1, 1, n) if red == "none" else torch.tensor([0.75])
+    loss, lse = flce.ce_forward(z, labels.to(dev), mask=m, reduction=red, num_label_tokens=nlt)
+    dz = flce.ce_backward(z, labels.to(dev), lse, grad.to(dev), mask=m, reduction=red,
+                          num_label_tokens=nlt)
+    torch.cuda.synchronize(dev)
+    zf = full[:, :v].double().numpy()
+    mk = mask.numpy() if mask is not None else None
+    ref = O.ce_forward(zf, labels.numpy(), mask=mk, reduction=red, num_label_tokens=nlt)
+    rdz = O.ce_backward(zf, labels.numpy(), mask=mk, reduction=red, num_label_tokens=nlt,
+                        grad_loss=grad.double().numpy())
+    got = {"loss": loss.double().cpu().numpy(), "lse": lse.double().cpu().numpy(),
+           "dh": dz.double().cpu().numpy(), "dw": np.zeros(1), "status": flce.get_error(dev)}
+    assert_parity(got, {"loss": np.asarray(ref.loss), "lse": ref.lse, "dh": rdz,
+                        "dw": np.zeros(1)}), c
