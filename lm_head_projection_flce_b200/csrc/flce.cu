@@ -39,6 +39,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>  // header-only; ranges cost a pointer test unless a tool attaches
+
 #include "flce.h"
 #include "epilogues.cuh"
 #include "gemm_sm100.cuh"
@@ -346,9 +348,20 @@ static cudaEvent_t take_event(int dev) {
   return e;
 }
 
+// An NVTX range over a host-side scope (an entry point, one launch), so a
+// profiler's timeline and its kernel filters can attribute GPU work.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 class LaunchScope {
  public:
-  LaunchScope(int family, double flops, double bytes, cudaStream_t st) : st_(st) {
+  LaunchScope(int family, double flops, double bytes, cudaStream_t st)
+      : st_(st), range_(kFamilyNames[family]) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     std::lock_guard<std::mutex> lock(g_prof_mutex);
     if (!g_prof_on) return;
@@ -370,6 +383,7 @@ class LaunchScope {
 
  private:
   cudaStream_t st_;
+  NvtxRange range_;
   ProfRecord rec_{};
   bool active_ = false;
 };
@@ -670,6 +684,7 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
                             int64_t unpadded, int64_t ignore_index, float softcap, int reduction,
                             int64_t num_label_tokens, float* loss, float* lse, void* workspace,
                             size_t ws_bytes, flce_stream_t stream) {
+  NvtxRange range("flce_forward");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
   int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
                         num_label_tokens);
@@ -747,6 +762,7 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
                              int reduction, int64_t num_label_tokens, const float* grad_loss,
                              const float* lse, void* dhidden, void* dweight, void* workspace,
                              size_t ws_bytes, flce_stream_t stream) {
+  NvtxRange range("flce_backward");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
   int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
                         num_label_tokens);
@@ -1056,6 +1072,7 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
                                     int64_t unpadded, int64_t ignore_index, float softcap,
                                     int reduction, int64_t num_label_tokens, float* loss,
                                     float* lse, flce_stream_t stream) {
+  NvtxRange range("flce_forward_noalloc");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
   if (!shape_ok(n, h, vp, v, w_dtype)) return FLCE_ERR_INVALID_ARG;
   // The whole scratch must fit the fixed array; nothing here can grow it.
@@ -1174,6 +1191,7 @@ extern "C" int flce_ce_forward(const void* logits, int dtype, const int64_t* lab
                                int64_t ignore_index, int reduction, int64_t num_label_tokens,
                                float* loss, float* lse, void* workspace, size_t ws_bytes,
                                flce_stream_t stream) {
+  NvtxRange range("flce_ce_forward");
   int st = check_ce(logits, dtype, labels, n, v, ld, reduction, num_label_tokens);
   if (st != FLCE_OK) return st;
   if ((n > 0 || reduction != FLCE_NONE) && (loss == nullptr || !aligned(loss, 4)))
@@ -1233,6 +1251,7 @@ extern "C" int flce_ce_backward(const void* logits, int dtype, const int64_t* la
                                 int64_t ignore_index, int reduction, int64_t num_label_tokens,
                                 const float* grad_loss, const float* lse, void* dlogits,
                                 void* workspace, size_t ws_bytes, flce_stream_t stream) {
+  NvtxRange range("flce_ce_backward");
   int st = check_ce(logits, dtype, labels, n, v, ld, reduction, num_label_tokens);
   if (st != FLCE_OK) return st;
   if (n > 0) {
