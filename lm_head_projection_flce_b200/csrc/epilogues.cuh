@@ -58,11 +58,13 @@ struct EpiForward {
     const int64_t ylocal = y - vbase;
     const int ncols = static_cast<int>(min(static_cast<int64_t>(kBN), p.vocab - vbase));
     float m = -INFINITY, s = 0.0f, zl = 0.0f;
+    const bool capped = p.softcap > 0.0f;
+    const float2 l2e = make_float2(kLog2e, kLog2e);
 #pragma unroll 1
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_load_32cols(taddr + c0, v);
-      if (p.softcap > 0.0f) {
+      if (capped) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = softcap_value(v[j], p.softcap, p.softcap_k);
       }
@@ -80,19 +82,33 @@ struct EpiForward {
         for (int j = 0; j < 2; ++j) t2[j] = (jl & 2) ? t4[j + 2] : t4[j];
         zl = (jl & 1) ? t2[1] : t2[0];
       }
-      float cmax = -INFINITY;
+      if (c0 + 32 > ncols) {  // only in the vocabulary's last tile
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float u = (c0 + j < ncols) ? v[j] * kLog2e : -INFINITY;
-        v[j] = u;
-        cmax = fmaxf(cmax, u);
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j >= ncols) v[j] = -INFINITY;
       }
-      const float mn = fmaxf(m, cmax);
-      if (mn != -INFINITY) {
-        float acc = 0.0f;
+      // max on the raw values (log2 e > 0 keeps the order), then
+      // 2^(z log2 e - mn) with the scale folded into one packed FMA per pair.
+      float c[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc += fast_exp2(v[j] - mn);
-        s = s * fast_exp2(m - mn) + acc;
+      for (int j = 0; j < 16; ++j) c[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) c[j] = fmaxf(c[j], c[j + w]);
+      const float mn = fmaxf(m, c[0] * kLog2e);
+      if (mn != -INFINITY) {
+        const float2 nm = make_float2(-mn, -mn);
+        float2 a0 = make_float2(0.0f, 0.0f), a1 = a0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float2 t0 = __ffma2_rn(make_float2(v[j], v[j + 1]), l2e, nm);
+          const float2 t1 = __ffma2_rn(make_float2(v[j + 2], v[j + 3]), l2e, nm);
+          a0 = __fadd2_rn(a0, make_float2(fast_exp2(t0.x), fast_exp2(t0.y)));
+          a1 = __fadd2_rn(a1, make_float2(fast_exp2(t1.x), fast_exp2(t1.y)));
+        }
+        const float2 a = __fadd2_rn(a0, a1);
+        s = s * fast_exp2(m - mn) + (a.x + a.y);
         m = mn;
       }
     }
@@ -134,18 +150,41 @@ struct EpiGrad {
     const float sc = live ? p.scale[n] : 0.0f;
     const int ncols = static_cast<int>(min(static_cast<int64_t>(kBN), p.vocab - vbase));
     uint4* out = reinterpret_cast<uint4*>(p.g + (live ? n : 0) * p.ldg + static_cast<int64_t>(nt) * kBN);
+    const bool capped = p.softcap > 0.0f;
+    const float2 l2e = make_float2(kLog2e, kLog2e), nl2 = make_float2(-l2, -l2),
+                 sc2 = make_float2(sc, sc);
 #pragma unroll 1
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_load_32cols(taddr + c0, v);
+      if (!capped) {
+        // sc * 2^(z log2 e - lse log2 e), two columns per packed FMA / multiply
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        float zc = v[j], dcap = 1.0f;
-        if (p.softcap > 0.0f) zc = softcap_value_grad(v[j], p.softcap, p.softcap_k, dcap);
-        const float prob = fast_exp2(zc * kLog2e - l2);
-        const float onehot = (c0 + j == ylocal) ? 1.0f : 0.0f;
-        const float gr = (prob - onehot) * dcap * sc;
-        v[j] = (c0 + j < ncols) ? gr : 0.0f;
+        for (int j = 0; j < 32; j += 2) {
+          const float2 t = __ffma2_rn(make_float2(v[j], v[j + 1]), l2e, nl2);
+          const float2 g = __fmul2_rn(make_float2(fast_exp2(t.x), fast_exp2(t.y)), sc2);
+          v[j] = g.x;
+          v[j + 1] = g.y;
+        }
+        if (ylocal >= c0 && ylocal < c0 + 32) {  // the label's column: - sc
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j == ylocal) v[j] -= sc;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float dcap;
+          const float zc = softcap_value_grad(v[j], p.softcap, p.softcap_k, dcap);
+          const float prob = fast_exp2(zc * kLog2e - l2);
+          const float onehot = (c0 + j == ylocal) ? 1.0f : 0.0f;
+          v[j] = (prob - onehot) * dcap * sc;
+        }
+      }
+      if (c0 + 32 > ncols) {  // only in the vocabulary's last tile
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j >= ncols) v[j] = 0.0f;
       }
       if (live) {
 #pragma unroll
