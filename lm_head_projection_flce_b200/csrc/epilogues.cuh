@@ -13,17 +13,17 @@ namespace flce {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Softcap c*tanh(z/c) from tanh(x) = 1 - 2/(exp(2x) + 1); also returns
-// d(c*tanh(z/c))/dz = 1 - tanh^2 = 4r(1-r) with r = 1/(exp(2x)+1), which stays
-// finite at both ends (r -> 0 and r -> 1).  k = 2*log2(e)/c.
-__device__ __forceinline__ float softcap_value(float z, float c, float k) {
-  const float r = fast_rcp(fast_exp2(z * k) + 1.0f);
-  return c - 2.0f * c * r;
-}
-__device__ __forceinline__ float softcap_value_grad(float z, float c, float k, float& dcap) {
-  const float r = fast_rcp(fast_exp2(z * k) + 1.0f);
-  dcap = 4.0f * r * (1.0f - r);
-  return c - 2.0f * c * r;
+// Softcap c*tanh(z/c) from tanh(x) = 1 - 2/(exp(2x) + 1), on two columns at
+// once with packed FP32 arithmetic: zc = c - 2c r with r = 1/(2^(z k) + 1),
+// k = 2*log2(e)/c.  r is returned for the derivative
+// d(c*tanh(z/c))/dz = 1 - tanh^2 = 4r(1-r), which stays finite at both ends
+// (r -> 0 and r -> 1).  c2 = (c, c), m2c = (-2c, -2c), k2 = (k, k).
+__device__ __forceinline__ float2 softcap_pair(float2 z, float2 c2, float2 m2c, float2 k2,
+                                               float2& r) {
+  const float2 t = __fmul2_rn(z, k2);
+  const float2 e = __fadd2_rn(make_float2(fast_exp2(t.x), fast_exp2(t.y)), make_float2(1.0f, 1.0f));
+  r = make_float2(fast_rcp(e.x), fast_rcp(e.y));
+  return __ffma2_rn(r, m2c, c2);  // c - 2c r
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -65,8 +65,16 @@ struct EpiForward {
       float v[32];
       tmem_load_32cols(taddr + c0, v);
       if (capped) {
+        const float2 c2 = make_float2(p.softcap, p.softcap);
+        const float2 m2c = make_float2(-2.0f * p.softcap, -2.0f * p.softcap);
+        const float2 k2 = make_float2(p.softcap_k, p.softcap_k);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = softcap_value(v[j], p.softcap, p.softcap_k);
+        for (int j = 0; j < 32; j += 2) {
+          float2 r;
+          const float2 zc = softcap_pair(make_float2(v[j], v[j + 1]), c2, m2c, k2, r);
+          v[j] = zc.x;
+          v[j + 1] = zc.y;
+        }
       }
       if (ylocal >= c0 && ylocal < c0 + 32) {
         // Pick column ylocal - c0 with a select tree on its bits (no local-memory indexing).
@@ -172,13 +180,32 @@ struct EpiGrad {
             if (c0 + j == ylocal) v[j] -= sc;
         }
       } else {
+        // (2^(zc log2 e - lse log2 e) - onehot) * sc * 4r(1 - r), two columns at a time
+        const float2 c2 = make_float2(p.softcap, p.softcap);
+        const float2 m2c = make_float2(-2.0f * p.softcap, -2.0f * p.softcap);
+        const float2 k2 = make_float2(p.softcap_k, p.softcap_k);
+        const float2 four = make_float2(4.0f, 4.0f);
+        auto pair = [&](int j, bool label) {
+          float2 r;
+          const float2 zc = softcap_pair(make_float2(v[j], v[j + 1]), c2, m2c, k2, r);
+          const float2 q = __fmul2_rn(r, four);
+          const float2 dsc = __fmul2_rn(__ffma2_rn(make_float2(-q.x, -q.y), r, q), sc2);
+          const float2 t = __ffma2_rn(zc, l2e, nl2);
+          float2 pr = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          if (label) {
+            if (c0 + j == ylocal) pr.x -= 1.0f;
+            if (c0 + j + 1 == ylocal) pr.y -= 1.0f;
+          }
+          const float2 g = __fmul2_rn(pr, dsc);
+          v[j] = g.x;
+          v[j + 1] = g.y;
+        };
+        if (ylocal >= c0 && ylocal < c0 + 32) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float dcap;
-          const float zc = softcap_value_grad(v[j], p.softcap, p.softcap_k, dcap);
-          const float prob = fast_exp2(zc * kLog2e - l2);
-          const float onehot = (c0 + j == ylocal) ? 1.0f : 0.0f;
-          v[j] = (prob - onehot) * dcap * sc;
+          for (int j = 0; j < 32; j += 2) pair(j, true);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) pair(j, false);
         }
       }
       if (c0 + 32 > ncols) {  // only in the vocabulary's last tile
