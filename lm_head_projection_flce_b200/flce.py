@@ -285,6 +285,68 @@ def fused_linear_cross_entropy(hidden, weight, labels, *, ignore_index: int = -1
                                 reduction, num_label_tokens)
 
 
+class CapturedStep:
+    """Forward + backward of the fused loss captured once into a CUDA graph.
+
+    The inputs are static device tensors owned here (``hidden``, ``labels``,
+    and the head ``weight`` the caller passes, which must stay alive and keep
+    its storage); a step copies new values into them (``set_inputs``) and
+    calls ``replay()``, which reruns all of the step's kernel launches as one
+    graph launch.  Outputs (``loss``, ``lse``, ``dhidden``, ``dweight``) are static
+    too and are overwritten by each replay.  Worth it where a step is short
+    enough for launch overhead to show (small batches); the results equal the
+    eager calls bit for bit.
+    """
+
+    def __init__(self, hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
+                 unpadded_vocab: int | None = None, reduction: str = "sum",
+                 num_label_tokens: int | None = None, grad_loss=None):
+        hid, lab = _prepare(hidden, weight, labels)
+        dev = hid.device
+        n, h = hid.shape
+        self.hidden = hid.clone()
+        self.labels = lab.clone()
+        self.weight = weight
+        self.kw = dict(ignore_index=ignore_index, softcap=softcap, unpadded_vocab=unpadded_vocab,
+                       reduction=reduction, num_label_tokens=num_label_tokens)
+        v = _vocab(weight, unpadded_vocab)
+        self.workspace = torch.empty(max(workspace_size(n, h, weight.shape[0], v, weight.dtype), 16),
+                                     dtype=torch.uint8, device=dev)
+        self.loss = torch.empty(n if reduction == "none" else 1, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(n, dtype=torch.float32, device=dev)
+        self.dhidden = torch.empty_like(self.hidden)
+        self.dweight = torch.empty_like(weight)
+        g = torch.ones(()) if grad_loss is None else grad_loss
+        self.grad = _grad_loss(g, n, reduction, dev).clone()
+        stream = torch.cuda.Stream(dev)
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            self._step()          # eager: per-device set-up and launch shapes, outside capture
+        torch.cuda.current_stream(dev).wait_stream(stream)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            self._step()
+
+    def _step(self):
+        forward(self.hidden, self.weight, self.labels, loss=self.loss, lse=self.lse,
+                workspace=self.workspace, **self.kw)
+        backward(self.hidden, self.weight, self.labels, self.lse, self.grad,
+                 dhidden=self.dhidden, dweight=self.dweight, workspace=self.workspace, **self.kw)
+
+    def set_inputs(self, hidden=None, labels=None) -> None:
+        """Copy new token data into the captured input buffers (same shapes)."""
+        if hidden is not None:
+            self.hidden.copy_(hidden.reshape(self.hidden.shape), non_blocking=True)
+        if labels is not None:
+            self.labels.copy_(labels.reshape(self.labels.shape), non_blocking=True)
+
+    def replay(self):
+        """Run forward + backward; returns (loss, dhidden, dweight), static buffers."""
+        self.graph.replay()
+        loss = self.loss if self.kw["reduction"] == "none" else self.loss.reshape(())
+        return loss, self.dhidden, self.dweight
+
+
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(load_library().flce_launch_count())

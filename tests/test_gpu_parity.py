@@ -378,3 +378,28 @@ def test_fp32_head_chunkings_noalloc_and_graph_replay(dev):
         for a, b in zip(eager, (loss, lse, dh, dw)):
             assert torch.equal(a, b)
     assert flce.get_error(dev) == flce.FLCE_OK
+
+
+def test_captured_step_replays_the_eager_step(dev):
+    """flce.CapturedStep: a forward + backward captured into a CUDA graph over
+    static buffers equals the eager calls bit for bit, also after new token
+    data is copied into its input buffers."""
+    w = CASES["ktail_softcap_padded"]
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab)
+
+    def eager(h, y):
+        loss, lse = flce.forward(h, wt, y, **kw)
+        dh, dw = flce.backward(h, wt, y, lse, torch.ones(1, device=dev), **kw)
+        return loss, dh, dw
+
+    step = flce.CapturedStep(hid, wt, lab, **kw)
+    for h, y in ((hid, lab), (hid.flip(0).contiguous(), lab.roll(7).contiguous())):
+        step.set_inputs(h, y)
+        got = [t.clone() for t in step.replay()]
+        ref = eager(h, y)
+        torch.cuda.synchronize(dev)
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+    assert flce.get_error(dev) == flce.FLCE_OK
