@@ -1,8 +1,8 @@
 """FP64 CPU oracle for the fused LM-head projection + cross-entropy.
 
 TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
-only the tests, the package smoke check and the benchmark's CPU-baseline leg
-call it.  It shares no code, constant or helper with the CUDA path; the two
+only the tests, the package smoke check and the benchmark's CPU-baseline and
+reference (``--impl reference``) legs call it.  It shares no code, constant or helper with the CUDA path; the two
 meet only in the seeded input generators, which hold none of the arithmetic.
 
 What is computed, and where the pages fix it:
