@@ -403,3 +403,35 @@ def test_captured_step_replays_the_eager_step(dev):
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
     assert flce.get_error(dev) == flce.FLCE_OK
+
+
+@pytest.mark.parametrize("name", ["tiny_n64_h256_v1024", "n4096_h4096_v128256"])
+def test_matches_torch_cross_entropy_on_fp32_logits(dev, name):
+    """Library cross-check ("matching PyTorch behavior"): with no softcap and
+    V = Vp, torch's cross_entropy and autograd on the FP32 logits of the same
+    BF16 inputs give the loss, dhidden and dW of the fused kernels, which never
+    form those logits.  The 64-token and the benchmark workload (the latter
+    in the launch configuration bench.py times)."""
+    w = W.WORKLOADS[name]
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    nlt = d["num_label_tokens"] if w.normalize_by_label_tokens else None
+    loss, lse = flce.forward(hid, wt, lab, reduction=w.reduction, num_label_tokens=nlt)
+    dh, dw = flce.backward(hid, wt, lab, lse, torch.ones(1, device=dev), reduction=w.reduction,
+                           num_label_tokens=nlt)
+    h32 = hid.float().requires_grad_(True)
+    w32 = wt.float().requires_grad_(True)
+    z = h32 @ w32.T
+    ref = torch.nn.functional.cross_entropy(z, lab, ignore_index=W.IGNORE_INDEX, reduction="sum")
+    if nlt:
+        ref = ref / nlt
+    ref.backward()
+    ref_lse = torch.logsumexp(z.detach(), dim=1)
+    torch.cuda.synchronize(dev)
+    assert flce.get_error(dev) == flce.FLCE_OK
+    assert float((lse - ref_lse).abs().max()) <= LSE_ABS
+    r = float(ref.detach())
+    assert abs(float(loss) - r) <= 1e-4 * abs(r)
+    for got, want in ((dh.float(), h32.grad), (dw.float(), w32.grad)):
+        scale = float(want.abs().max())
+        assert float((got - want).abs().max()) <= GRAD_REL * scale
