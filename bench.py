@@ -41,7 +41,7 @@ METRIC = "fused linear-CE fwd+bwd tokens/sec on 1 B200; % of dense-BF16 tensor p
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "n4096_h4096_v128256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.md")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_per_launch.json")
 
 
 def parse_args(argv=None):
@@ -52,6 +52,11 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the short timed passes of the other large workloads and of cross "
+                         "entropy on given logits (one GPU only) under 'extra_workloads'")
+    ap.add_argument("--extra-steps", type=int, default=5,
+                    help="timed steps of each extra workload (at least 5)")
     ap.add_argument("--path", choices=["flce", "chunked_ce"], default="flce",
                     help="flce: the fused projection + CE (default); chunked_ce: cross entropy "
                          "on given logits [4096, 128256] BF16")
@@ -85,20 +90,21 @@ def kernel_source_digest() -> str:
 
 
 def committed_traffic(workload: str, family: str) -> float | None:
-    """DRAM bytes per launch of `family` from the committed ncu summary, if it was
-    taken on the current kernel sources and this workload; else None."""
+    """DRAM bytes per launch of `family` on `workload` from the committed ncu
+    record (profiles/dram_traffic_per_launch.json), if it was taken on the
+    current kernel sources; else None."""
     try:
-        text = open(PROFILE_TRAFFIC).read()
-    except OSError:
+        with open(PROFILE_TRAFFIC) as f:
+            records = json.load(f)["records"]
+    except (OSError, ValueError, KeyError, TypeError):
         return None
     digest = kernel_source_digest()
-    for line in text.splitlines():
-        # | family | workload | source digest | dram bytes per launch | ...
-        cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) >= 4 and cells[0] == family and cells[1] == workload and cells[2] == digest:
+    for r in records:
+        if (r.get("family") == family and r.get("workload") == workload
+                and r.get("source_digest") == digest):
             try:
-                return float(cells[3])
-            except ValueError:
+                return float(r["bytes_per_launch"])
+            except (KeyError, TypeError, ValueError):
                 return None
     return None
 
@@ -299,6 +305,195 @@ def run_reference(args, w) -> int:
 
 # ------------------------------------------------------------------ GPU path
 
+def tensor_roofline(stats: dict, peaks: dict, peak_src: str, workload: str,
+                    whole_path_flops: float, whole_path_ms: float) -> dict:
+    """Roofline of the dominant contraction (the kernel family with the most device
+    time): algorithmic FLOPs / its CUDA-event time against the measured dense-BF16
+    peak.  The denominator is the burst cuBLAS figure -- the bench's timed
+    regions are a fraction of a second to a few seconds, the regime that figure
+    was taken in; the sustained (power-capped, seconds-long loop) figure is
+    reported beside it.  A fraction above 1 means the timed kernel did not do the
+    work it claims, so it is refused (frac null) rather than reported."""
+    gemms = {k: v for k, v in stats.items() if v["flops"] > 0}
+    name = max(gemms, key=lambda k: gemms[k]["total_ms"])
+    dom = gemms[name]
+    achieved = dom["flops"] / (dom["total_ms"] / 1e3) / 1e12
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    whole = whole_path_flops / (whole_path_ms / 1e3) / 1e12
+    out = {
+        "bound": "tensor", "kernel": name, "achieved": achieved, "peak": burst,
+        "unit": "TFLOP/s", "frac": achieved / burst,
+        "traffic": committed_traffic(workload, name),
+        "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + write.sum)",
+        "flops_per_launch": dom["flops"] / dom["launches"],
+        "launches": dom["launches"],
+        "peak_source": f"{peak_src} bf16_tflops (cuBLAS dense BF16, burst)",
+        "peak_sustained": sustained, "frac_of_sustained": achieved / sustained,
+        "whole_path_tflops": whole, "whole_path_frac": whole / burst,
+    }
+    if out["frac"] > 1.0 or out["whole_path_frac"] > 1.0:
+        out["frac_refused"] = (f"{out['frac']:.3f} / {out['whole_path_frac']:.3f} of the burst "
+                               "peak: above 1, so the timing does not cover the work claimed")
+        out["frac"] = None
+        out["whole_path_frac"] = None
+    return out
+
+
+def hbm_roofline(stats: dict, peaks: dict, peak_src: str, workload: str, prefix: str) -> dict:
+    """Roofline of the dominant single-pass HBM kernel: algorithmic bytes / time
+    against the measured copy bandwidth (refused above 1, as for the GEMMs)."""
+    hbm = {k: v for k, v in stats.items() if v["bytes"] > 0 and k.startswith(prefix)}
+    name = max(hbm, key=lambda k: hbm[k]["total_ms"])
+    dom = hbm[name]
+    achieved = dom["bytes"] / (dom["total_ms"] / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    out = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
+           "frac": achieved / peak, "traffic": committed_traffic(workload, name),
+           "bytes_per_launch": dom["bytes"] / dom["launches"],
+           "peak_source": f"{peak_src} hbm_gbs (copy read+write)"}
+    if out["frac"] > 1.0:
+        out["frac_refused"] = f"{out['frac']:.3f} of the copy bandwidth: above 1"
+        out["frac"] = None
+    return out
+
+
+def kernel_table(stats: dict, steps: int) -> dict:
+    return {k: {"launches_per_step": st["launches"] / steps,
+                "ms_per_step": st["total_ms"] / steps,
+                **({"tflops": st["flops"] / (st["total_ms"] / 1e3) / 1e12} if st["flops"] > 0 else
+                   {"gbs": st["bytes"] / (st["total_ms"] / 1e3) / 1e9 if st["total_ms"] > 0
+                    else None})}
+            for k, st in sorted(stats.items())}
+
+
+class Timer:
+    """Device timing of `steps` calls of `step` on `stream`: CUDA events on the
+    launching stream around the whole region (barrier + synchronize on both
+    sides) and between steps, the library's launch count, optionally its
+    per-launch events, and nvidia-smi clock samples taken meanwhile."""
+
+    def __init__(self, dev, stream, uuid, barrier=lambda: None):
+        self.dev, self.stream, self.uuid, self.barrier = dev, stream, uuid, barrier
+
+    def run(self, step, steps: int, profile: bool = False):
+        import torch
+        from lm_head_projection_flce_b200 import flce
+        sampler = ClockSampler(self.uuid)
+        sampler.start()
+        self.barrier()
+        torch.cuda.synchronize(self.dev)
+        if profile:
+            flce.profile_start()
+        l0 = flce.launch_count()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(self.stream)
+        for k in range(steps):
+            step()
+            ev[k + 1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        self.barrier()
+        launches = flce.launch_count() - l0
+        stats = flce.profile_stop() if profile else {}
+        clocks = sampler.stop()
+        per_step = [ev[k].elapsed_time(ev[k + 1]) for k in range(steps)]
+        return {"ms": ev[0].elapsed_time(ev[steps]), "per_step": per_step,
+                "launches": launches, "stats": stats, "clocks": clocks}
+
+
+class FlceRun:
+    """One workload's inputs, outputs and workspace on the device, and its step:
+    forward + backward through the binding, the backward reusing the forward's
+    BF16 copy of an FP32 head (same workspace, head unchanged in between)."""
+
+    def __init__(self, w, dev, graph: bool = False):
+        import torch
+        from lm_head_projection_flce_b200 import flce
+        from lm_head_projection_flce_b200 import workloads as W
+        self.w = w
+        self.data = W.generate(w)           # seeded on the CPU: the same batch on every rank
+        d = self.data
+        self.hid = d["hidden"].to(dev)
+        self.wt = d["weight"].to(dev)
+        self.lab = d["labels"].to(dev)
+        n, h, vp, v = w.n_tokens, w.hidden, w.padded_vocab, w.vocab
+        self.nlt = d["num_label_tokens"] if w.normalize_by_label_tokens else None
+        self.ws = torch.empty(flce.workspace_size(n, h, vp, v, self.wt.dtype), dtype=torch.uint8,
+                              device=dev)
+        self.loss = torch.empty(1, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(n, dtype=torch.float32, device=dev)
+        self.dh = torch.empty_like(self.hid)
+        self.dw = torch.empty_like(self.wt)
+        self.grad = torch.ones(1, dtype=torch.float32, device=dev)
+        self.kw = dict(softcap=w.softcap, unpadded_vocab=v, reduction=w.reduction,
+                       num_label_tokens=self.nlt, workspace=self.ws)
+        self.reuse = self.wt.dtype == torch.float32
+        self.captured = None
+        self.graph_launches = 0
+        if graph:
+            l0 = flce.launch_count()
+            self.captured = flce.CapturedStep(self.hid, self.wt, self.lab, softcap=w.softcap,
+                                              unpadded_vocab=v, reduction=w.reduction,
+                                              num_label_tokens=self.nlt)
+            self.graph_launches = (flce.launch_count() - l0) // 2  # eager set-up + capture
+            self.loss = self.captured.loss
+
+    def step(self, h_in=None, l_in=None):
+        from lm_head_projection_flce_b200 import flce
+        if self.captured is not None:
+            if h_in is not None:
+                self.captured.set_inputs(h_in, l_in)
+            self.captured.replay()
+            return
+        h_in = self.hid if h_in is None else h_in
+        l_in = self.lab if l_in is None else l_in
+        flce.forward(h_in, self.wt, l_in, loss=self.loss, lse=self.lse, **self.kw)
+        flce.backward(h_in, self.wt, l_in, self.lse, self.grad, dhidden=self.dh, dweight=self.dw,
+                      reuse_head_copy=self.reuse, **self.kw)
+
+
+def measure_flce(run: "FlceRun", timer: "Timer", steps: int, warmup: int, world: int,
+                 max_over_ranks, peaks, peak_src) -> dict:
+    """Warm-up, the headline pass (no per-launch events), a re-measure if any
+    rank saw a hardware/thermal slowdown, then a profiled pass for the kernels."""
+    import torch
+    from lm_head_projection_flce_b200 import flce
+    dev = timer.dev
+    for _ in range(warmup):
+        run.step()
+    torch.cuda.synchronize(dev)
+    status = flce.get_error(dev)
+    if status != flce.FLCE_OK:
+        raise RuntimeError(f"device error during warm-up: {flce.STATUS[status]}")
+    head = timer.run(run.step, steps)
+    remeasured = False
+    # The decision is collective so every rank takes the same barriers.
+    bad = 1.0 if BAD_REASONS & set(head["clocks"].get("reasons", [])) else 0.0
+    if max_over_ranks(bad) > 0:
+        head = timer.run(run.step, steps)
+        remeasured = True
+    prof = timer.run(run.step, steps, profile=True) if run.captured is None else None
+    if flce.get_error(dev) != flce.FLCE_OK:
+        raise RuntimeError("device error word set during the timed region")
+    ms_max = max_over_ranks(head["ms"])
+    w = run.w
+    path_flops = w.flops_fwd_bwd * steps
+    if prof is not None:
+        roof = tensor_roofline(prof["stats"], peaks, peak_src, w.name, path_flops, ms_max)
+        kernels = kernel_table(prof["stats"], steps)
+        launches = head["launches"]
+    else:  # graph replays carry no per-launch events: the whole step is the unit
+        stats = {"whole step (CUDA graph replay)": {
+            "flops": path_flops, "total_ms": ms_max, "launches": run.graph_launches * steps,
+            "bytes": 0.0}}
+        roof = tensor_roofline(stats, peaks, peak_src, w.name, path_flops, ms_max)
+        kernels = {}
+        launches = run.graph_launches * steps
+    return {"ms": ms_max, "per_step": head["per_step"], "launches": launches,
+            "clocks": {**head["clocks"], "remeasured": remeasured}, "roofline": roof,
+            "kernels": kernels}
+
+
 def run_ours(args, w) -> int:
     import torch
     import torch.distributed as dist
@@ -326,100 +521,30 @@ def run_ours(args, w) -> int:
     from lm_head_projection_flce_b200 import build as B
     B.build()                               # no-op when the in-tree library matches its sources
     flce.load_library()
-    d = W.generate(w)                       # seeded on the CPU: the same batch on every rank
-    hid = d["hidden"].to(dev)
-    wt = d["weight"].to(dev)
-    lab = d["labels"].to(dev)
-    n, h, vp, v = w.n_tokens, w.hidden, w.padded_vocab, w.vocab
-    nlt = d["num_label_tokens"] if w.normalize_by_label_tokens else None
-    ws = torch.empty(flce.workspace_size(n, h, vp, v, wt.dtype), dtype=torch.uint8, device=dev)
-    loss = torch.empty(1, dtype=torch.float32, device=dev)
-    lse = torch.empty(n, dtype=torch.float32, device=dev)
-    dh = torch.empty_like(hid)
-    dw = torch.empty_like(wt)
-    grad = torch.ones(1, dtype=torch.float32, device=dev)
-    kw = dict(softcap=w.softcap, unpadded_vocab=v, reduction=w.reduction, num_label_tokens=nlt,
-              workspace=ws)
-
-    def step(h_in=hid, l_in=lab):
-        flce.forward(h_in, wt, l_in, loss=loss, lse=lse, **kw)
-        flce.backward(h_in, wt, l_in, lse, grad, dhidden=dh, dweight=dw, **kw)
-
-    captured = None
-    if args.graph:
-        l0 = flce.launch_count()
-        captured = flce.CapturedStep(hid, wt, lab, softcap=w.softcap, unpadded_vocab=v,
-                                     reduction=w.reduction, num_label_tokens=nlt)
-        graph_launches = (flce.launch_count() - l0) // 2  # the eager set-up step + the capture
-        loss = captured.loss
-
-        def step(h_in=None, l_in=None):  # noqa: F811 - the graph replaces the eager calls
-            if h_in is not None:
-                captured.set_inputs(h_in, l_in)
-            captured.replay()
-
-    warmup = max(args.warmup, 3)
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    status = flce.get_error(dev)
-    if status != flce.FLCE_OK:
-        raise RuntimeError(f"device error during warm-up: {flce.STATUS[status]}")
-
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         uuid = None
     stream = torch.cuda.current_stream(dev)
+    timer = Timer(dev, stream, uuid, barrier)
+    peaks, peak_src = load_peaks()
+    warmup = max(args.warmup, 3)
 
-    def timed_region(profile: bool):
-        sampler = ClockSampler(uuid)
-        sampler.start()
-        barrier()
-        torch.cuda.synchronize(dev)
-        if profile:
-            flce.profile_start()
-        l0 = flce.launch_count()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        launches = flce.launch_count() - l0
-        stats = flce.profile_stop() if profile else {}
-        clocks = sampler.stop()
-        return e0.elapsed_time(e1), launches, stats, clocks
-
-    # The headline pass runs without per-launch events (a few microseconds per
-    # launch, which shows on small workloads); the per-kernel figures of the
-    # roofline come from a second pass of the same steps with the events on.
-    ms, launches, _, clocks = timed_region(False)
-    remeasured = False
-    # Re-measure once if any rank saw a hardware or thermal slowdown; the
-    # decision is collective so every rank takes the same barriers.
-    bad = 1.0 if BAD_REASONS & set(clocks.get("reasons", [])) else 0.0
-    if max_over_ranks(bad) > 0:
-        ms, launches, _, clocks = timed_region(False)
-        remeasured = True
-    stats = timed_region(True)[2] if captured is None else {}
-    if captured is not None:  # replays enqueue no library call: count the graph's kernels
-        launches = graph_launches * args.steps
-    ms_max = max_over_ranks(ms)
-    if flce.get_error(dev) != flce.FLCE_OK:
-        raise RuntimeError("device error word set during the timed region")
+    run = FlceRun(w, dev, graph=args.graph)
+    m = measure_flce(run, timer, args.steps, warmup, world, max_over_ranks, peaks, peak_src)
+    n = w.n_tokens
+    value = aggregate_throughput(n, args.steps, world, m["ms"])
 
     # ---- end to end: pinned host inputs -> device, fwd + bwd, loss -> host, every step.
     # Step k+1's inputs are copied on a second stream into the other of two
     # device buffers while step k computes; every copy is inside the timed
     # region (the copy stream starts after e0, the last step waits for its copy).
+    d = run.data
     h_host = d["hidden"].pin_memory()
     l_host = d["labels"].pin_memory()
     loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
     copy_stream = torch.cuda.Stream(dev)
-    bufs = [(torch.empty_like(hid), torch.empty_like(lab)) for _ in range(2)]
+    bufs = [(torch.empty_like(run.hid), torch.empty_like(run.lab)) for _ in range(2)]
     copied = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]
 
@@ -440,9 +565,9 @@ def run_ours(args, w) -> int:
                 stage(k + 1)
             b = k % 2
             stream.wait_event(copied[b])
-            step(*bufs[b])
+            run.step(*bufs[b])
             consumed[b].record(stream)
-            loss_host.copy_(loss, non_blocking=True)
+            loss_host.copy_(run.loss, non_blocking=True)
 
     e2e_run(2)
     barrier()
@@ -455,66 +580,62 @@ def run_ours(args, w) -> int:
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-
-    value = aggregate_throughput(n, args.steps, world, ms_max)
     e2e_value = aggregate_throughput(n, args.steps, world, e2e_ms)
+    h2d = run.hid.numel() * run.hid.element_size() + run.lab.numel() * 8
 
-    peaks, peak_src = load_peaks()
-    gemms = {k: s for k, s in stats.items() if s["flops"] > 0}
-    if captured is None:
-        dom_name = max(gemms, key=lambda k: gemms[k]["total_ms"])
-        dom = gemms[dom_name]
-    else:  # graph replays carry no per-launch events: the whole step is the unit
-        dom_name = "whole step (CUDA graph replay)"
-        dom = {"flops": w.flops_fwd_bwd * args.steps, "total_ms": ms_max,
-               "launches": graph_launches * args.steps}
-    achieved = dom["flops"] / (dom["total_ms"] / 1e3) / 1e12
-    # The kernels are timed inside a seconds-long continuous run (clocks settle
-    # under the power cap), so the sustained GEMM figure is the denominator;
-    # the burst figure is reported beside it.
-    peak_burst = float(peaks["bf16_tflops"])
-    peak = float(peaks.get("bf16_tflops_sustained", peak_burst))
-    per_step_launches = dom["launches"] / args.steps
-    traffic = committed_traffic(w.name, dom_name)
-    kernels = {k: {"launches_per_step": s["launches"] / args.steps,
-                   "ms_per_step": s["total_ms"] / args.steps,
-                   **({"tflops": s["flops"] / (s["total_ms"] / 1e3) / 1e12} if s["flops"] > 0 else
-                      {"gbs": s["bytes"] / (s["total_ms"] / 1e3) / 1e9 if s["total_ms"] > 0 else None})}
-               for k, s in sorted(stats.items())}
-    path_flops = w.flops_fwd_bwd * args.steps * world
-
+    line = None
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "warmup": warmup, "ms_per_step": m["ms"] / args.steps,
+            "ms_per_step_median": statistics.median(m["per_step"]),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**workload_config(w, f"replicas x{world} (one independent batch per GPU)"),
-                       **({"cuda_graph": True} if captured is not None else {})},
-            "roofline": {
-                "bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + write.sum)",
-                "flops_per_launch": dom["flops"] / dom["launches"],
-                "launches_per_step": per_step_launches,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS, seconds-long loop)",
-                "peak_burst": peak_burst, "frac_of_burst": achieved / peak_burst,
-                "whole_path_tflops": path_flops / (ms_max / 1e3) / 1e12 / world,
-                "whole_path_frac": path_flops / (ms_max / 1e3) / 1e12 / world / peak,
-                "whole_path_frac_of_burst": path_flops / (ms_max / 1e3) / 1e12 / world / peak_burst,
-            },
-            "kernels": kernels,
+                       **({"cuda_graph": True} if args.graph else {})},
+            "roofline": m["roofline"],
+            "kernels": m["kernels"],
             "kernel_timing": ("per-launch CUDA events in a second pass of the same steps"
-                              if captured is None else "none inside a CUDA graph"),
-            "e2e": {"value": e2e_value, "unit": UNIT,
-                    "h2d_bytes_per_step": hid.numel() * hid.element_size() + lab.numel() * 8,
+                              if not args.graph else "none inside a CUDA graph"),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": 4,
                     "api": "lm_head_projection_flce_b200.flce.forward/backward (C ABI via ctypes)",
                     "overlap": "step k+1's H2D copy on a second stream during step k"},
-            "gpu_launches": launches,
-            "clocks": {**clocks, "remeasured": remeasured},
+            "gpu_launches": m["launches"],
+            "clocks": m["clocks"],
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, d)
+    del bufs, h_host, l_host, run
+    torch.cuda.empty_cache()
+
+    # ---- the other large workloads and cross entropy on given logits, one GPU only:
+    # a short timed pass each, reported under their own key (the headline stays above).
+    if world == 1 and not args.no_extras and not args.graph:
+        extras = {}
+        for wx in (W.SOFTCAP_F32_HEAD, W.LONG_SEQ, W.LARGE_HEAD):
+            if wx.name == w.name:
+                continue
+            rx = FlceRun(wx, dev)
+            k = max(5, args.extra_steps)
+            mx = measure_flce(rx, timer, k, 3, 1, lambda x: x, peaks, peak_src)
+            entry = {"value": wx.n_tokens * k / (mx["ms"] / 1e3), "unit": UNIT, "steps": k,
+                     "warmup": 3, "ms_per_step": mx["ms"] / k,
+                     "ms_per_step_median": statistics.median(mx["per_step"]),
+                     "config": workload_config(wx, "one GPU"), "roofline": mx["roofline"],
+                     "kernels": mx["kernels"], "gpu_launches": mx["launches"],
+                     "clocks": mx["clocks"]}
+            if not args.no_cpu_baseline:
+                entry["cpu_baseline"] = cpu_baseline(wx, rx.data, target_s=6.0)
+            extras[wx.name] = entry
+            del rx
+            torch.cuda.empty_cache()
+        extras[W.CE_LOGITS.name] = measure_chunked_ce(
+            timer, max(5, args.extra_steps), 3, peaks, peak_src,
+            with_cpu_baseline=not args.no_cpu_baseline)
+        line["extra_workloads"] = extras
+
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         barrier()
@@ -522,20 +643,38 @@ def run_ours(args, w) -> int:
     return 0
 
 
-def run_chunked_ce(args) -> int:
-    """Cross entropy on given logits: forward + backward per step (HBM-bound)."""
+def ce_cpu_baseline(d: dict, target_s: float = 6.0) -> dict:
+    """The oracle's cross entropy on given logits, timed on a token sample."""
+    import numpy as np
     import torch
+    from oracle import flce_oracle as O
+    z = d["logits"]
+    lab = d["labels"].numpy()
+    rng = np.random.default_rng(7)
+    s = 16
+    while True:
+        rows = np.sort(rng.choice(z.shape[0], size=s, replace=False))
+        zs = z[torch.from_numpy(rows)].double().numpy()
+        t0 = time.perf_counter()
+        O.ce_forward(zs, lab[rows])
+        O.ce_backward(zs, lab[rows])
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or s >= z.shape[0]:
+            break
+        s = min(4 * s, z.shape[0])
+    return {"value": s / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"{s} seeded token rows of the logits through the FP64 oracle's cross "
+                       f"entropy forward + backward, {dt:.1f} s (the FP64 upcast of the rows "
+                       "excluded)")}
 
+
+def measure_chunked_ce(timer: "Timer", steps: int, warmup: int, peaks, peak_src,
+                       with_cpu_baseline: bool) -> dict:
+    """Cross entropy on given logits [4096, 128256] BF16: forward + backward per step."""
+    import torch
     from lm_head_projection_flce_b200 import flce
     from lm_head_projection_flce_b200 import workloads as W
-
-    if not torch.cuda.is_available():
-        raise RuntimeError("bench.py needs a CUDA device (sm_100a)")
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
-    from lm_head_projection_flce_b200 import build as B
-    B.build()
-    flce.load_library()
+    dev = timer.dev
     w = W.CE_LOGITS
     d = W.generate_logits(w)
     z = d["logits"].to(dev)
@@ -546,78 +685,72 @@ def run_chunked_ce(args) -> int:
                      device=dev)
     dz = torch.empty_like(z)
     grad = torch.ones(1, device=dev)
+    loss = torch.empty(1, device=dev)
+    lse = torch.empty(n, device=dev)
 
-    def step(z_in=z, l_in=lab):
-        loss, lse = flce.ce_forward(z_in, l_in, reduction=w.reduction, num_label_tokens=nlt,
-                                    workspace=ws)
-        flce.ce_backward(z_in, l_in, lse, grad, reduction=w.reduction, num_label_tokens=nlt,
+    def step():
+        flce.ce_forward(z, lab, reduction=w.reduction, num_label_tokens=nlt, workspace=ws,
+                        loss=loss, lse=lse)
+        flce.ce_backward(z, lab, lse, grad, reduction=w.reduction, num_label_tokens=nlt,
                          dlogits=dz, workspace=ws)
-        return loss
 
-    warmup = max(args.warmup, 3)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
-    stream = torch.cuda.current_stream(dev)
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        uuid = None
-    def timed(profile: bool):
-        torch.cuda.synchronize(dev)
-        if profile:
-            flce.profile_start()
-        l0 = flce.launch_count()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        launches = flce.launch_count() - l0
-        stats = flce.profile_stop() if profile else None
-        return e0.elapsed_time(e1), launches, stats
-
     # The steps here are ~0.5 ms, so the per-launch events of the kernel
     # profile would add a few percent: the step time comes from a pass
     # without them, the per-kernel figures from a second, profiled pass.
-    sampler = ClockSampler(uuid)
-    sampler.start()
-    ms, launches, _ = timed(False)
-    _, _, stats = timed(True)
-    clocks = sampler.stop()
+    head = timer.run(step, steps)
+    prof = timer.run(step, steps, profile=True)
     if flce.get_error(dev) != flce.FLCE_OK:
         raise RuntimeError("device error word set during the timed region")
-    peaks, peak_src = load_peaks()
-    hbm = [k for k, st in stats.items() if st["bytes"] > 0 and k.startswith("ce_logits")]
-    dom_name = max(hbm, key=lambda k: stats[k]["total_ms"])
-    dom = stats[dom_name]
-    achieved = dom["bytes"] / (dom["total_ms"] / 1e3) / 1e9
-    peak = float(peaks["hbm_gbs"])
-    line = {
+    out = {
         "metric": "cross entropy on given logits, fwd+bwd tokens/sec on 1 B200",
-        "value": n * args.steps / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "value": n * steps / (head["ms"] / 1e3), "unit": UNIT, "steps": steps, "warmup": warmup,
+        "ms_per_step": head["ms"] / steps, "ms_per_step_median": statistics.median(head["per_step"]),
+        "dtype": "bf16",
         "config": {"workload": w.name, "n_tokens": n, "vocab": v, "logits_dtype": w.dtype,
                    "logits_sigma": w.sigma, "ignore_frac": w.ignore_frac,
                    "reduction": "sum/num_label_tokens",
                    "l2": "inputs larger than L2: 1.05 GB of logits read twice and 1.05 GB of "
                          "gradient written every step"},
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": committed_traffic(w.name, dom_name),
-                     "bytes_per_launch": dom["bytes"] / dom["launches"],
-                     "peak_source": f"{peak_src} hbm_gbs (copy read+write)"},
-        "kernels": {k: {"launches_per_step": st["launches"] / args.steps,
-                        "ms_per_step": st["total_ms"] / args.steps,
-                        "gbs": st["bytes"] / (st["total_ms"] / 1e3) / 1e9 if st["total_ms"] > 0 else None}
-                    for k, st in sorted(stats.items())},
+        "roofline": hbm_roofline(prof["stats"], peaks, peak_src, w.name, "ce_logits"),
+        "kernels": kernel_table(prof["stats"], steps),
         "kernel_timing": "per-launch CUDA events in a second pass of the same steps",
-        "gpu_launches": launches,
-        "clocks": clocks,
+        "gpu_launches": head["launches"],
+        "clocks": head["clocks"],
     }
+    if with_cpu_baseline:
+        out["cpu_baseline"] = ce_cpu_baseline(d)
+    del z, dz, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_chunked_ce(args) -> int:
+    """--path chunked_ce: cross entropy on given logits as the headline line."""
+    import torch
+
+    from lm_head_projection_flce_b200 import flce
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device (sm_100a)")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    from lm_head_projection_flce_b200 import build as B
+    B.build()
+    flce.load_library()
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    timer = Timer(dev, torch.cuda.current_stream(dev), uuid)
+    peaks, peak_src = load_peaks()
+    m = measure_chunked_ce(timer, args.steps, max(args.warmup, 3), peaks, peak_src,
+                           with_cpu_baseline=not args.no_cpu_baseline)
+    line = {"metric": m.pop("metric"), "value": m.pop("value"), "unit": UNIT, "n_gpus": 1,
+            **m, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "data": "synthetic"}
     print(json.dumps(line), flush=True)
     return 0
 

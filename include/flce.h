@@ -128,6 +128,33 @@ int flce_backward(const void* hidden, const void* weight, int w_dtype, const int
                   void* workspace, size_t ws_bytes, flce_stream_t stream);
 
 /*
+ * flce_backward with option flags.  The pages compute the head's BF16 copy
+ * once per step (inkling2 page, Inkling2FusedLinearCrossEntropy class
+ * docstring: an FP32 head is rounded to BF16, "the cast FSDP applies", and the
+ * gradient flows back through that cast); this lets the backward reuse the
+ * copy the forward made instead of casting again.
+ *   flags  0, or FLCE_BWD_HEAD_COPY_VALID: the caller promises that the first
+ *          V*H*2 bytes of `workspace` (rounded up to 1 KiB) still hold the BF16
+ *          copy of weight[:V] that flce_forward wrote there -- the forward ran
+ *          on this workspace with this weight pointer, shape and w_dtype, and
+ *          neither the head nor those workspace bytes changed since.  The
+ *          backward then skips its own FP32 -> BF16 cast of the head (one read
+ *          of V*H*4 bytes and one write of V*H*2).  The flag is ignored for a
+ *          BF16 head, which is used in place.  The library cannot check the
+ *          promise: a stale copy gives wrong gradients without an error.
+ *          Any other bit set: FLCE_ERR_INVALID_ARG.
+ * flce_backward(...) is flce_backward_ex(..., 0, stream).
+ */
+#define FLCE_BWD_HEAD_COPY_VALID 1u
+int flce_backward_ex(const void* hidden, const void* weight, int w_dtype,
+                     const int64_t* labels, int64_t n_tokens, int64_t hidden_size,
+                     int64_t padded_vocab, int64_t unpadded_vocab, int64_t ignore_index,
+                     float softcap, int reduction, int64_t num_label_tokens,
+                     const float* grad_loss, const float* lse, void* dhidden, void* dweight,
+                     void* workspace, size_t ws_bytes, unsigned int flags,
+                     flce_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the calling device's error word:
  * FLCE_ERR_BAD_LABEL if a kernel saw a label outside [0, V) that was not
  * ignore_index, FLCE_ERR_TIMEOUT if a pipeline wait gave up (the affected
@@ -204,7 +231,7 @@ int flce_ce_backward(const void* logits, int dtype, const int64_t* labels, const
  *   forward scratch (8 B x ceil(V/256) x N for the logsumexp partials, plus
  *   4 B x N, plus the BF16 copy of an FP32 head) exceeds 32 MiB is refused
  *   with FLCE_ERR_WORKSPACE and nothing is enqueued; e.g. N = 4096 tokens with
- *   V = 128256 and a BF16 head needs 16.5 MiB and fits.
+ *   V = 128256 and a BF16 head needs 15.7 MiB (16.4 MB) and fits.
  *   The array is shared by every call on a device and keeps whatever the last
  *   call left in it; the forward writes every scratch byte before reading it,
  *   so nothing has to be cleared between calls.  Calls that overlap on the GPU
@@ -212,7 +239,9 @@ int flce_ce_backward(const void* logits, int dtype, const int64_t* labels, const
  *   them on one stream or synchronise between them.
  *   The first call on each device looks up the array's device address with
  *   cudaGetSymbolAddress (with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is looked up again whenever the
+ *   device's CUDA context has changed (after cudaDeviceReset, for instance),
+ *   so that call too belongs outside a capture.
  */
 int flce_forward_noalloc(const void* hidden, const void* weight, int w_dtype,
                          const int64_t* labels, int64_t n_tokens, int64_t hidden_size,

@@ -60,15 +60,9 @@ constexpr size_t kAlign = 1024;
 constexpr size_t kChunkBudgetBytes = size_t(1) << 30;  // default cap on each G buffer
 constexpr int64_t kMinChunk = 4096;
 
-// Contractions run on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2) unless
-// built with FLCE_SINGLE_CTA (one CTA per 128 x 256 tile).
-#ifdef FLCE_SINGLE_CTA
-constexpr bool kUsePairs = false;
-#else
-constexpr bool kUsePairs = true;
-#endif
-constexpr int kTileRows = kUsePairs ? kPairBM : kBM;      // output rows per tile
-constexpr int kBBoxRows = kUsePairs ? kBN / 2 : kBN;      // K-major B rows loaded per CTA
+// Contractions run on CTA pairs: 256 x 256 tiles, tcgen05 cta_group::2.
+constexpr int kTileRows = kPairBM;   // output rows per tile
+constexpr int kBBoxRows = kBN / 2;   // K-major B rows loaded per CTA (half of the tile's)
 
 // ------------------------------------------------------------------ kernels
 
@@ -261,6 +255,7 @@ __global__ void wait_timeout_selftest_kernel(unsigned* err, uint64_t timeout_ns)
 
 struct DeviceInfo {
   bool init = false;
+  unsigned long long ctx_id = 0;  // driver id of the context the cached addresses belong to
   int status = FLCE_OK;
   int num_sms = 0;
   int max_pairs = 0;  // CTA pairs of the pair GEMM that fit at once (0 = not yet queried)
@@ -272,13 +267,43 @@ static std::mutex g_mutex;
 static DeviceInfo g_dev[64];
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Id of the calling thread's current CUDA context, 0 when it has none (for
+// instance right after cudaDeviceReset, until the runtime creates a new one).
+// Device addresses looked up in one context (the error word, the no-allocation
+// scratch array) are stale in the next, so they are cached with this id.
+static unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 static int device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FLCE_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& d = g_dev[dev];
+  if (d.init && (ctx == 0 || ctx != d.ctx_id)) d.init = false;  // a new context: look up again
   if (!d.init) {
     d.init = true;
+    d.status = FLCE_OK;
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -300,6 +325,8 @@ static int device_info(DeviceInfo** out) {
       else
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    // The lookups above made the runtime create the context if it had none.
+    d.ctx_id = current_context_id();
   }
   if (d.status != FLCE_OK) {
     d.init = false;  // retry next call (e.g. after the caller fixed the device)
@@ -453,6 +480,7 @@ static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool
   p.epi = epi;
   p.num_kb = int(cdiv(k, kBK));
   p.raster = make_raster(m, n, k);
+  p.a_keep = p.raster.n_fast ? 0 : 1;  // the grouped operand's panels are the reused ones
   p.tiles = (m > 0 && n > 0) ? int64_t(p.raster.m_tiles) * p.raster.n_tiles : 0;
   return p;
 }
@@ -483,57 +511,47 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   g.tile_counter = counter;
   g.err = dev.err;
   g.timeout_ns = kDefaultTimeoutNs;
-  if constexpr (kUsePairs) {
-    auto kern = tc_gemm_pair_kernel<EpiSet<kKinds>, C0, C1, C2>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kPairSmemBytes)) != cudaSuccess)
-      return FLCE_ERR_CUDA;
-    // Pairs that can be resident at once (clusters need two SMs of one GPC);
-    // queried once per device (every instantiation shares the launch shape).
-    int max_pairs = dev.max_pairs;
-    if (max_pairs == 0) {
-      cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * (dev.num_sms / 2), 1, 1);
-      q.blockDim = dim3(kThreads, 1, 1);
-      q.dynamicSmemBytes = kPairSmemBytes;
-      cudaLaunchAttribute qa[1];
-      qa[0].id = cudaLaunchAttributeClusterDimension;
-      qa[0].val.clusterDim.x = 2;
-      qa[0].val.clusterDim.y = 1;
-      qa[0].val.clusterDim.z = 1;
-      q.attrs = qa;
-      q.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0)
-        n = dev.num_sms / 2;
-      max_pairs = std::min(n, dev.num_sms / 2);
-      std::lock_guard<std::mutex> lock(g_mutex);
-      dev.max_pairs = max_pairs;
-    }
-    const int pairs = int(std::min<int64_t>(max_pairs, total));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kPairSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    LaunchScope scope(family, flops, bytes, st);
-    if (cudaLaunchKernelEx(&cfg, kern, maps, g, ep) != cudaSuccess) return FLCE_ERR_CUDA;
-  } else {
-    auto kern = tc_gemm_group_kernel<EpiSet<kKinds>, C0, C1, C2>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kGemmSmemBytes)) != cudaSuccess)
-      return FLCE_ERR_CUDA;
-    const int grid = int(std::min<int64_t>(dev.num_sms, total));
-    LaunchScope scope(family, flops, bytes, st);
-    kern<<<grid, kThreads, kGemmSmemBytes, st>>>(maps, g, ep);
+  auto kern = tc_gemm_pair_kernel<EpiSet<kKinds>, C0, C1, C2>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(kPairSmemBytes)) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  // Pairs that can be resident at once (clusters need two SMs of one GPC);
+  // queried once per device (every instantiation shares the launch shape).
+  int max_pairs = dev.max_pairs;
+  if (max_pairs == 0) {
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2 * (dev.num_sms / 2), 1, 1);
+    q.blockDim = dim3(kThreads, 1, 1);
+    q.dynamicSmemBytes = kPairSmemBytes;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0)
+      n = dev.num_sms / 2;
+    max_pairs = std::min(n, dev.num_sms / 2);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    dev.max_pairs = max_pairs;
   }
+  const int pairs = int(std::min<int64_t>(max_pairs, total));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LaunchScope scope(family, flops, bytes, st);
+  if (cudaLaunchKernelEx(&cfg, kern, maps, g, ep) != cudaSuccess) return FLCE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
@@ -575,17 +593,24 @@ struct BwdPlan {
   size_t off_lse2, off_scale, off_cnt, off_dh32, off_wb, off_g, fixed, total;
 };
 
+// Both plans put the BF16 copy of an FP32 head at offset 0, so a backward
+// given the forward's workspace finds the copy the forward wrote there
+// (flce_backward_ex with FLCE_BWD_HEAD_COPY_VALID).
+static size_t head_copy_bytes(const Shape& s) {
+  return s.w_dtype == FLCE_F32 ? align_up(size_t(s.v) * s.h * 2) : 0;
+}
+
 static FwdPlan plan_forward(const Shape& s) {
   FwdPlan p{};
   p.v_tiles = cdiv(s.v, kBN);
   p.nblk = cdiv(s.n, kMergeRows);
-  size_t o = 0;
+  p.off_wb = 0;
+  size_t o = head_copy_bytes(s);
   p.off_pm = o;  o = align_up(o + size_t(p.v_tiles) * s.n * 4);
   p.off_ps = o;  o = align_up(o + size_t(p.v_tiles) * s.n * 4);
   p.off_zl = o;  o = align_up(o + size_t(s.n) * 4);
   p.off_bl = o;  o = align_up(o + size_t(p.nblk) * 8);
   p.off_bc = o;  o = align_up(o + size_t(p.nblk) * 4);
-  p.off_wb = o;  o = align_up(o + (s.w_dtype == FLCE_F32 ? size_t(s.v) * s.h * 2 : 0));
   p.total = std::max(o, kAlign);  // never zero, so N = 0 still has a valid buffer
   return p;
 }
@@ -600,13 +625,13 @@ static int64_t default_chunk(const Shape& s) {
 static BwdPlan plan_backward(const Shape& s, int64_t vc) {
   BwdPlan p{};
   p.vc = vc;
-  size_t o = 0;
+  p.off_wb = 0;
+  size_t o = head_copy_bytes(s);
   p.off_lse2 = o;  o = align_up(o + size_t(s.n) * 4);
   p.off_scale = o; o = align_up(o + size_t(s.n) * 4);
   p.n_counters = cdiv(s.v, kBN) + 2;  // one per launch at the narrowest chunking
   p.off_cnt = o;   o = align_up(o + size_t(p.n_counters) * 4);
   p.off_dh32 = o;  o = align_up(o + size_t(s.n) * s.h * 4);
-  p.off_wb = o;    o = align_up(o + (s.w_dtype == FLCE_F32 ? size_t(s.v) * s.h * 2 : 0));
   p.fixed = o;
   p.off_g = o;     o = align_up(o + 2 * size_t(s.n) * vc * 2);  // two chunk buffers
   p.total = o;
@@ -756,17 +781,18 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   return FLCE_OK;
 }
 
-extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype,
-                             const int64_t* labels, int64_t n, int64_t h, int64_t vp,
-                             int64_t unpadded, int64_t ignore_index, float softcap,
-                             int reduction, int64_t num_label_tokens, const float* grad_loss,
-                             const float* lse, void* dhidden, void* dweight, void* workspace,
-                             size_t ws_bytes, flce_stream_t stream) {
+extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dtype,
+                                const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                                int64_t unpadded, int64_t ignore_index, float softcap,
+                                int reduction, int64_t num_label_tokens, const float* grad_loss,
+                                const float* lse, void* dhidden, void* dweight, void* workspace,
+                                size_t ws_bytes, unsigned int flags, flce_stream_t stream) {
   NvtxRange range("flce_backward");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
   int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
                         num_label_tokens);
   if (st != FLCE_OK) return st;
+  if ((flags & ~FLCE_BWD_HEAD_COPY_VALID) != 0u) return FLCE_ERR_INVALID_ARG;
   if (dweight == nullptr || !aligned(dweight, 16)) return FLCE_ERR_INVALID_ARG;
   if (n > 0) {
     if (grad_loss == nullptr || lse == nullptr || dhidden == nullptr) return FLCE_ERR_INVALID_ARG;
@@ -802,9 +828,12 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
   const void* wb = weight;
   if (w_dtype == FLCE_F32) {
     wb = ws + p.off_wb;
-    if ((st = launch_cast(static_cast<const float*>(weight),
+    // The caller vouches that the copy at offset 0 still holds bf16(weight[:V])
+    // (written by flce_forward on this workspace and unchanged since).
+    if ((flags & FLCE_BWD_HEAD_COPY_VALID) == 0u &&
+        (st = launch_cast(static_cast<const float*>(weight),
                           reinterpret_cast<__nv_bfloat16*>(ws + p.off_wb), v * h, *dev, cs)) !=
-        FLCE_OK)
+            FLCE_OK)
       return st;
   }
   float* lse2 = reinterpret_cast<float*>(ws + p.off_lse2);
@@ -923,6 +952,17 @@ extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype
       return st;
   }
   return FLCE_OK;
+}
+
+extern "C" int flce_backward(const void* hidden, const void* weight, int w_dtype,
+                             const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                             int64_t unpadded, int64_t ignore_index, float softcap,
+                             int reduction, int64_t num_label_tokens, const float* grad_loss,
+                             const float* lse, void* dhidden, void* dweight, void* workspace,
+                             size_t ws_bytes, flce_stream_t stream) {
+  return flce_backward_ex(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index,
+                          softcap, reduction, num_label_tokens, grad_loss, lse, dhidden, dweight,
+                          workspace, ws_bytes, 0u, stream);
 }
 
 extern "C" int flce_get_error(flce_stream_t stream) {
@@ -1064,6 +1104,7 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB on every de
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 static std::mutex g_noalloc_mutex;
 static void* g_noalloc_addr[64];  // device address of g_noalloc_scratch, per device
+static unsigned long long g_noalloc_ctx[64];  // context that address belongs to
 
 }  // namespace flce
 
@@ -1082,15 +1123,18 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FLCE_ERR_CUDA;
   void* scratch = nullptr;
   {
-    // First call on a device: look up where the array lives on it.  In host
-    // code the array's name is only a host-side stand-in, never a device
-    // address, so the kernels get this looked-up pointer instead.
+    // First call on a device (or in a new context on it, e.g. after
+    // cudaDeviceReset): look up where the array lives.  In host code the
+    // array's name is only a host-side stand-in, never a device address, so
+    // the kernels get this looked-up pointer instead.
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_addr[dev] == nullptr) {
+    if (g_noalloc_addr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
         return FLCE_ERR_CUDA;
       g_noalloc_addr[dev] = p;
+      g_noalloc_ctx[dev] = current_context_id();
     }
     scratch = g_noalloc_addr[dev];
   }

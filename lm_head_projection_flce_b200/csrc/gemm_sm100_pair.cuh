@@ -38,10 +38,13 @@ __device__ __forceinline__ bool pair_produce_tile(const GemmProblem& pr, const C
                                                   uint32_t rank, uint32_t smem_base,
                                                   uint32_t bar_base, uint32_t leader_bar_base,
                                                   int& stage, uint32_t& phase, PipeCtl* ctl,
-                                                  const GemmGroup& g) {
+                                                  const GemmGroup& g, uint64_t pol_keep,
+                                                  uint64_t pol_stream, bool reverse_k) {
   const int am = mt * kPairBM + 128 * static_cast<int>(rank) + pr.a_mn_off;
   const int bm = nt * kBN + 128 * static_cast<int>(rank) + pr.b_mn_off;
   const int num_kb = pr.num_kb;
+  const uint64_t pol_a = pr.a_keep ? pol_keep : pol_stream;
+  const uint64_t pol_b = pr.a_keep ? pol_stream : pol_keep;
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_phase(bar_base + 8u * (kPairStages + stage), phase ^ 1u, ctl, g.err, g.timeout_ns))
       return false;
@@ -50,20 +53,24 @@ __device__ __forceinline__ bool pair_produce_tile(const GemmProblem& pr, const C
     const uint32_t fb = leader_bar_base + 8u * stage;
     const uint32_t sa = smem_base + stage * kPairStageBytes;
     const uint32_t sb = sa + kPairATileBytes;
-    const int kc = kb * kBK;
+    // Serpentine: odd waves of tiles walk K downwards, so they start on the
+    // k-blocks the previous wave read last, which are still in L2.  The MMA
+    // side is unchanged: it consumes stages in order and zero-initialises the
+    // accumulator on the first one, whichever k-block that holds.
+    const int kc = (reverse_k ? num_kb - 1 - kb : kb) * kBK;
     if constexpr (!C::kAMn) {
-      tma_load_2d_pair(sa, ma, fb, kc + pr.a_k_off, am);
+      tma_load_2d_pair_hint(sa, ma, fb, kc + pr.a_k_off, am, pol_a);
     } else {
 #pragma unroll
       for (int j = 0; j < 2; ++j)
-        tma_load_2d_pair(sa + j * kMnBlockBytes, ma, fb, am + 64 * j, kc + pr.a_k_off);
+        tma_load_2d_pair_hint(sa + j * kMnBlockBytes, ma, fb, am + 64 * j, kc + pr.a_k_off, pol_a);
     }
     if constexpr (!C::kBMn) {
-      tma_load_2d_pair(sb, mb, fb, kc + pr.b_k_off, bm);
+      tma_load_2d_pair_hint(sb, mb, fb, kc + pr.b_k_off, bm, pol_b);
     } else {
 #pragma unroll
       for (int j = 0; j < 2; ++j)
-        tma_load_2d_pair(sb + j * kMnBlockBytes, mb, fb, bm + 64 * j, kc + pr.b_k_off);
+        tma_load_2d_pair_hint(sb + j * kMnBlockBytes, mb, fb, bm + 64 * j, kc + pr.b_k_off, pol_b);
     }
     if (++stage == kPairStages) {
       stage = 0;
@@ -197,6 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return c >= g.total_tiles ? -1 : c;
       };
+      const uint64_t pol_keep = l2_policy_evict_last();
+      const uint64_t pol_stream = l2_policy_evict_first();
       int64_t claimed = rank == 0 ? claim() : -1;
       while (ok) {
         int64_t t;
@@ -227,16 +236,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const GemmProblem& pr = g.prob[p];
         int mt, nt;
         pr.raster.coords(t - pr.tile_begin, mt, nt);
+        const bool rev = ((t / num_pairs) & 1) != 0;  // a function of the tile index only
         if (p == 0)
           ok = pair_produce_tile<C0>(pr, &maps.a[0], &maps.b[0], mt, nt, rank, smem_base, bar_base,
-                                     leader_bar_base, stage, phase, ctl, g);
+                                     leader_bar_base, stage, phase, ctl, g, pol_keep,
+                                     pol_stream, rev);
         else if constexpr (C1::kValid) {
           if (p == 1)
             ok = pair_produce_tile<C1>(pr, &maps.a[1], &maps.b[1], mt, nt, rank, smem_base,
-                                       bar_base, leader_bar_base, stage, phase, ctl, g);
+                                       bar_base, leader_bar_base, stage, phase, ctl, g,
+                                       pol_keep, pol_stream, rev);
           else if constexpr (C2::kValid)
             ok = pair_produce_tile<C2>(pr, &maps.a[2], &maps.b[2], mt, nt, rank, smem_base,
-                                       bar_base, leader_bar_base, stage, phase, ctl, g);
+                                       bar_base, leader_bar_base, stage, phase, ctl, g,
+                                       pol_keep, pol_stream, rev);
         }
       }
       if (!ok) {

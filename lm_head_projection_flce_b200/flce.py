@@ -33,6 +33,7 @@ STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_INVALID_ARG", 2: "FLCE_ERR_WORKSPACE",
           3: "FLCE_ERR_UNSUPPORTED", 4: "FLCE_ERR_CUDA", 5: "FLCE_ERR_BAD_LABEL",
           6: "FLCE_ERR_TIMEOUT"}
 REDUCTIONS = {"sum": 0, "mean": 1, "none": 2}
+FLCE_BWD_HEAD_COPY_VALID = 1
 W_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 _c_i64 = ctypes.c_int64
@@ -50,6 +51,10 @@ SIGNATURES = {
     "flce_backward": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
                                _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr,
                                _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "flce_backward_ex": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64,
+                                  _c_i64, _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr,
+                                  _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_size, ctypes.c_uint,
+                                  _c_ptr]),
     "flce_get_error": (_c_int, [_c_ptr]),
     "flce_status_string": (ctypes.c_char_p, [_c_int]),
     "flce_flops_fwd_bwd": (ctypes.c_double, [_c_i64, _c_i64, _c_i64]),
@@ -208,8 +213,15 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
              softcap: float = 0.0, unpadded_vocab: int | None = None, reduction: str = "sum",
              num_label_tokens: int | None = None, workspace: torch.Tensor | None = None,
              dhidden: torch.Tensor | None = None, dweight: torch.Tensor | None = None,
-             stream=None):
-    """Gradients ``(dhidden [.., H] bf16, dweight [Vp, H] in the head's dtype)``."""
+             reuse_head_copy: bool = False, stream=None):
+    """Gradients ``(dhidden [.., H] bf16, dweight [Vp, H] in the head's dtype)``.
+
+    ``reuse_head_copy=True`` (flce_backward_ex with FLCE_BWD_HEAD_COPY_VALID):
+    for an FP32 head, skip the FP32 -> BF16 cast and use the copy that
+    ``forward`` wrote into the same ``workspace`` -- the caller promises that
+    the head and that workspace are unchanged since.  Needs ``workspace``;
+    ignored for a BF16 head.
+    """
     lib = load_library()
     hid, lab = _prepare(hidden, weight, labels)
     n, h = hid.shape
@@ -223,11 +235,14 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
                else _buffer(dhidden, n * h, torch.bfloat16, dev, "dhidden"))
     dweight = (torch.empty_like(weight) if dweight is None
                else _buffer(dweight, weight.numel(), weight.dtype, dev, "dweight"))
+    if reuse_head_copy and workspace is None:
+        raise ValueError("reuse_head_copy needs the workspace the forward wrote the copy into")
     ws, ws_bytes = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
-    st = lib.flce_backward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
-                           v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
-                           _ptr(grad), _ptr(lse), _ptr(dhidden), _ptr(dweight), _ptr(ws),
-                           ws_bytes, _stream_handle(dev, stream))
+    flags = FLCE_BWD_HEAD_COPY_VALID if reuse_head_copy else 0
+    st = lib.flce_backward_ex(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h,
+                              vp, v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
+                              _ptr(grad), _ptr(lse), _ptr(dhidden), _ptr(dweight), _ptr(ws),
+                              ws_bytes, flags, _stream_handle(dev, stream))
     _check("flce_backward", st)
     return dhidden.reshape(hidden.shape), dweight
 
@@ -261,10 +276,20 @@ class _FusedLinearCE(torch.autograd.Function):
     @staticmethod
     def forward(ctx, hidden, weight, labels, ignore_index, softcap, unpadded_vocab, reduction,
                 num_label_tokens):
+        # An FP32 head's BF16 copy, made by the forward, is kept (in the
+        # workspace) for the backward instead of being cast again; autograd's
+        # version check refuses a backward after the head changed in place.
+        ws = None
+        if weight.dtype == torch.float32:
+            hid = hidden.reshape(-1, hidden.shape[-1])
+            need = workspace_size(hid.shape[0], hid.shape[1], weight.shape[0],
+                                  _vocab(weight, unpadded_vocab), weight.dtype)
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device=hidden.device)
         loss, lse = forward(hidden, weight, labels, ignore_index=ignore_index, softcap=softcap,
                             unpadded_vocab=unpadded_vocab, reduction=reduction,
-                            num_label_tokens=num_label_tokens)
+                            num_label_tokens=num_label_tokens, workspace=ws)
         ctx.save_for_backward(hidden, weight, labels, lse)
+        ctx.workspace = ws
         ctx.opts = (ignore_index, softcap, unpadded_vocab, reduction, num_label_tokens)
         return loss
 
@@ -272,8 +297,11 @@ class _FusedLinearCE(torch.autograd.Function):
     def backward(ctx, grad_out):
         hidden, weight, labels, lse = ctx.saved_tensors
         ii, c, uv, red, nlt = ctx.opts
+        ws = ctx.workspace
+        ctx.workspace = None
         dh, dw = backward(hidden, weight, labels, lse, grad_out, ignore_index=ii, softcap=c,
-                          unpadded_vocab=uv, reduction=red, num_label_tokens=nlt)
+                          unpadded_vocab=uv, reduction=red, num_label_tokens=nlt, workspace=ws,
+                          reuse_head_copy=ws is not None)
         return dh, dw, None, None, None, None, None, None
 
 
@@ -296,6 +324,14 @@ class CapturedStep:
     too and are overwritten by each replay.  Worth it where a step is short
     enough for launch overhead to show (small batches); the results equal the
     eager calls bit for bit.
+
+    The options, ``num_label_tokens`` included, are host values baked into
+    the graph when it is captured: a replay normalises by the count given at
+    construction even if ``set_inputs`` brought labels with another number of
+    live tokens.  ``set_inputs(..., num_label_tokens=k)`` refuses a ``k`` that
+    differs from the captured one; build a new CapturedStep for it.
+    An FP32 head is cast to BF16 once per replay (the backward reuses the
+    forward's copy).
     """
 
     def __init__(self, hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
@@ -331,10 +367,19 @@ class CapturedStep:
         forward(self.hidden, self.weight, self.labels, loss=self.loss, lse=self.lse,
                 workspace=self.workspace, **self.kw)
         backward(self.hidden, self.weight, self.labels, self.lse, self.grad,
-                 dhidden=self.dhidden, dweight=self.dweight, workspace=self.workspace, **self.kw)
+                 dhidden=self.dhidden, dweight=self.dweight, workspace=self.workspace,
+                 reuse_head_copy=self.weight.dtype == torch.float32, **self.kw)
 
-    def set_inputs(self, hidden=None, labels=None) -> None:
-        """Copy new token data into the captured input buffers (same shapes)."""
+    def set_inputs(self, hidden=None, labels=None, num_label_tokens: int | None = None) -> None:
+        """Copy new token data into the captured input buffers (same shapes).
+
+        ``num_label_tokens``, if given, must equal the value captured at
+        construction (it is fixed inside the graph); anything else raises.
+        """
+        if num_label_tokens is not None and num_label_tokens != self.kw["num_label_tokens"]:
+            raise ValueError(f"num_label_tokens={num_label_tokens} differs from the captured "
+                             f"{self.kw['num_label_tokens']}; it is fixed when the graph is "
+                             "captured")
         if hidden is not None:
             self.hidden.copy_(hidden.reshape(self.hidden.shape), non_blocking=True)
         if labels is not None:

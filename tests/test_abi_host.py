@@ -131,6 +131,25 @@ def test_bad_arguments_fail_closed_on_the_host(lib, call):
     assert call(lib, ws=FAKE + 8) == 2
 
 
+def test_backward_ex_flags(lib):
+    def bex(flags, **kw):
+        a = dict(hidden=FAKE, weight=FAKE, w_dtype=1, labels=FAKE, n=64, h=256, vp=1024, v=1024,
+                 ii=-100, c=0.0, red=0, nlt=0, grad=FAKE, lse=FAKE, dh=FAKE, dw=FAKE, ws=FAKE,
+                 ws_bytes=1 << 40, stream=None)
+        a.update(kw)
+        return lib.flce_backward_ex(a["hidden"], a["weight"], a["w_dtype"], a["labels"], a["n"],
+                                    a["h"], a["vp"], a["v"], a["ii"], a["c"], a["red"], a["nlt"],
+                                    a["grad"], a["lse"], a["dh"], a["dw"], a["ws"], a["ws_bytes"],
+                                    flags, a["stream"])
+    assert bex(2) == 1 and bex(0x80000000) == 1 and bex(3) == 1   # unknown bits
+    assert bex(1, h=250) == 1 and bex(1, ws=0) == 2              # the usual checks stay
+    # the documented flag passes the host checks (then the missing GPU answers)
+    import torch
+    if not torch.cuda.is_available():
+        assert bex(flce.FLCE_BWD_HEAD_COPY_VALID) in (3, 4)
+        assert bex(0) in (3, 4)
+
+
 def test_backward_specific_arguments(lib):
     for kw in (dict(grad=0), dict(lse=0), dict(dh=0), dict(dw=0), dict(dh=FAKE + 2),
                dict(dw=FAKE + 8)):

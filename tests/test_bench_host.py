@@ -100,11 +100,54 @@ def test_clock_summary():
 
 
 def test_committed_traffic_needs_matching_sources(tmp_path, monkeypatch):
-    f = tmp_path / "t.md"
+    f = tmp_path / "t.json"
     dig = bench.kernel_source_digest()
-    f.write_text("| family | workload | digest | bytes |\n|---|---|---|---|\n"
-                 f"| gemm_fwd_lse | w1 | {dig} | 123456 |\n| gemm_bwd_dw | w1 | 0000 | 7 |\n")
+    f.write_text(json.dumps({"records": [
+        {"family": "gemm_fwd_lse", "workload": "w1", "source_digest": dig,
+         "bytes_per_launch": 123456},
+        {"family": "gemm_bwd_dw", "workload": "w1", "source_digest": "0000",
+         "bytes_per_launch": 7}]}))
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(f))
     assert bench.committed_traffic("w1", "gemm_fwd_lse") == 123456.0
     assert bench.committed_traffic("w1", "gemm_bwd_dw") is None     # taken on other sources
     assert bench.committed_traffic("w2", "gemm_fwd_lse") is None
+    f.write_text("not json")
+    assert bench.committed_traffic("w1", "gemm_fwd_lse") is None
+
+
+def test_committed_traffic_record_is_well_formed():
+    with open(bench.PROFILE_TRAFFIC) as fh:
+        recs = json.load(fh)["records"]
+    for r in recs:
+        assert {"family", "workload", "source_digest", "bytes_per_launch", "command"} <= set(r)
+        assert r["bytes_per_launch"] > 0
+
+
+def _stats(ms_fwd, ms_bwd):
+    return {"gemm_fwd_lse": {"launches": 2, "total_ms": ms_fwd, "flops": 2e12, "bytes": 0.0},
+            "gemm_bwd_fused": {"launches": 12, "total_ms": ms_bwd, "flops": 12e12, "bytes": 0.0},
+            "lse_merge": {"launches": 2, "total_ms": 0.1, "flops": 0.0, "bytes": 1e8}}
+
+
+def test_tensor_roofline_uses_the_burst_peak_and_refuses_above_one():
+    peaks = {"bf16_tflops": 1650.0, "bf16_tflops_sustained": 1350.0}
+    r = bench.tensor_roofline(_stats(2.0, 10.0), peaks, "measured", "w", 16e12, 12.5)
+    assert r["kernel"] == "gemm_bwd_fused" and r["peak"] == 1650.0
+    assert r["achieved"] == pytest.approx(12e12 / 10e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1650.0)
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / 1350.0)
+    assert r["whole_path_frac"] == pytest.approx(16e12 / 12.5e-3 / 1e12 / 1650.0)
+    # a kernel 'faster' than the peak: the fraction is refused, not reported
+    fast = bench.tensor_roofline(_stats(0.5, 5.0), peaks, "measured", "w", 16e12, 5.0)
+    assert fast["frac"] is None and "frac_refused" in fast
+
+
+def test_hbm_roofline_refuses_above_one():
+    peaks = {"hbm_gbs": 6500.0}
+    st = {"ce_logits_fwd": {"launches": 1, "total_ms": 0.2, "flops": 0.0, "bytes": 1e9},
+          "ce_logits_bwd": {"launches": 1, "total_ms": 0.4, "flops": 0.0, "bytes": 2e9}}
+    r = bench.hbm_roofline(st, peaks, "measured", "w", "ce_logits")
+    assert r["kernel"] == "ce_logits_bwd" and r["frac"] == pytest.approx(5000.0 / 6500.0)
+    st["ce_logits_fwd"]["total_ms"] = 0.1
+    st["ce_logits_bwd"]["total_ms"] = 0.2     # 10000 GB/s: above the copy bandwidth
+    assert bench.hbm_roofline(st, peaks, "measured", "w", "ce_logits")["frac"] is None

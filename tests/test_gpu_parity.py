@@ -380,6 +380,62 @@ def test_fp32_head_chunkings_noalloc_and_graph_replay(dev):
     assert flce.get_error(dev) == flce.FLCE_OK
 
 
+def test_backward_reuses_the_forwards_head_copy(dev):
+    """flce_backward_ex with FLCE_BWD_HEAD_COPY_VALID: with an FP32 head the
+    backward skips its own cast and reads the BF16 copy the forward left at
+    the start of the workspace; dhidden and dW equal the recasting backward
+    bit for bit at every chunking, and one launch (the cast) is saved.  A
+    CapturedStep with an FP32 head (which uses the flag) and the autograd
+    wrapper (which keeps the forward's workspace) agree with them too."""
+    w = W.custom(300, 264, 5000, 5120, w_dtype="f32", softcap=30.0, ignore_frac=0.1, seed=23)
+    d = W.generate(w)
+    ref = run_oracle(d, w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab)
+    grad = torch.ones(1, device=dev)
+    lo = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, torch.float32,
+                             minimum=True)
+    hi = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, torch.float32)
+    for size in (lo, lo + 2 * w.n_tokens * 256 * 4, hi):
+        ws = torch.empty(size, dtype=torch.uint8, device=dev)
+        loss, lse = flce.forward(hid, wt, lab, workspace=ws, **kw)
+        l0 = flce.launch_count()
+        dh_a, dw_a = flce.backward(hid, wt, lab, lse, grad, workspace=ws, **kw)
+        l1 = flce.launch_count()
+        # clear the workspace: the flagged backward can then only see the
+        # copy that the next forward writes
+        ws.fill_(0xFF)
+        flce.forward(hid, wt, lab, workspace=ws, loss=loss, lse=lse, **kw)
+        l2 = flce.launch_count()
+        dh_b, dw_b = flce.backward(hid, wt, lab, lse, grad, workspace=ws, reuse_head_copy=True,
+                                   **kw)
+        l3 = flce.launch_count()
+        torch.cuda.synchronize(dev)
+        assert torch.equal(dh_a, dh_b) and torch.equal(dw_a, dw_b)
+        assert (l3 - l2) == (l1 - l0) - 1
+        got = {"loss": loss.double().cpu().numpy(), "lse": lse.double().cpu().numpy(),
+               "dh": dh_b.double().cpu().numpy(), "dw": dw_b.double().cpu().numpy(),
+               "status": flce.get_error(dev)}
+        assert_parity(got, ref)
+
+    step = flce.CapturedStep(hid, wt, lab, **kw)
+    loss_c, dh_c, dw_c = (t.clone() for t in step.replay())
+    torch.cuda.synchronize(dev)
+    assert torch.equal(dh_c, dh_a) and torch.equal(dw_c, dw_a)
+    with pytest.raises(ValueError):
+        step.set_inputs(hid, lab, num_label_tokens=7)
+
+    h = hid.clone().requires_grad_(True)
+    wr = wt.clone().requires_grad_(True)
+    flce.fused_linear_cross_entropy(h, wr, lab, **kw).backward()
+    torch.cuda.synchronize(dev)
+    assert torch.equal(h.grad, dh_a) and torch.equal(wr.grad, dw_a)
+    assert flce.get_error(dev) == flce.FLCE_OK
+
+    with pytest.raises(ValueError):   # the flag needs the forward's workspace
+        flce.backward(hid, wt, lab, lse, grad, reuse_head_copy=True, **kw)
+
+
 def test_captured_step_replays_the_eager_step(dev):
     """flce.CapturedStep: a forward + backward captured into a CUDA graph over
     static buffers equals the eager calls bit for bit, also after new token
