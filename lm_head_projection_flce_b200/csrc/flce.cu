@@ -480,7 +480,11 @@ static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool
   p.epi = epi;
   p.num_kb = int(cdiv(k, kBK));
   p.raster = make_raster(m, n, k);
-  p.a_keep = p.raster.n_fast ? 0 : 1;  // the grouped operand's panels are the reused ones
+  // Only an operand the raster holds whole in L2 (hidden, in the projection and
+  // recompute GEMMs and as dW's B) is worth protecting; a grouped panel of a
+  // larger operand is re-read only by tiles running at the same time.
+  p.a_keep = !p.raster.n_fast && p.raster.group == p.raster.m_tiles ? 1 : 0;
+  p.b_keep = p.raster.n_fast && p.raster.group == p.raster.n_tiles ? 1 : 0;
   p.tiles = (m > 0 && n > 0) ? int64_t(p.raster.m_tiles) * p.raster.n_tiles : 0;
   return p;
 }
@@ -584,7 +588,7 @@ struct Shape {
 
 struct FwdPlan {
   int64_t v_tiles, nblk;
-  size_t off_pm, off_ps, off_zl, off_bl, off_bc, off_wb, total;
+  size_t off_pm, off_ps, off_zl, off_bl, off_bc, off_cnt, off_wb, total;
 };
 
 struct BwdPlan {
@@ -611,6 +615,7 @@ static FwdPlan plan_forward(const Shape& s) {
   p.off_zl = o;  o = align_up(o + size_t(s.n) * 4);
   p.off_bl = o;  o = align_up(o + size_t(p.nblk) * 8);
   p.off_bc = o;  o = align_up(o + size_t(p.nblk) * 4);
+  p.off_cnt = o; o = align_up(o + 4);  // the projection GEMM's tile counter
   p.total = std::max(o, kAlign);  // never zero, so N = 0 still has a valid buffer
   return p;
 }
@@ -761,8 +766,12 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   ep.label_logit = reinterpret_cast<float*>(ws + p.off_zl);
   const double fwd_flops = 2.0 * double(n) * double(v) * double(h);
   const double fwd_bytes = 2.0 * (double(n) + double(v)) * double(h) + 8.0 * double(p.v_tiles) * n;
+  // Tiles are taken from a counter (zeroed here, in stream order), so pairs that
+  // run slower take fewer tiles and the launch does not wait on the slowest one.
+  unsigned* counter = reinterpret_cast<unsigned*>(ws + p.off_cnt);
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned), cs) != cudaSuccess) return FLCE_ERR_CUDA;
   if ((st = launch_group<kEpiSetForward, ProblemCfg<false, false, kEpiForward>>(
-           &prob, &ta, &tb, 1, es, nullptr, *dev, cs, KF_GEMM_FWD, fwd_flops, fwd_bytes)) !=
+           &prob, &ta, &tb, 1, es, counter, *dev, cs, KF_GEMM_FWD, fwd_flops, fwd_bytes)) !=
       FLCE_OK)
     return st;
   {

@@ -67,8 +67,8 @@ struct GemmProblem {
   int b_mn_off, b_k_off;  // offsets added to B's (MN, K) tile coordinates
   int epi;                // EpiKind
   int num_kb;             // ceil(k / kBK)
-  int a_keep;             // 1: A's panels are reused across the raster (keep A in L2, stream B);
-                          // 0: the other way round
+  int a_keep, b_keep;     // 1: the raster keeps all of this operand in L2 and every tile
+                          // row / column re-reads it: load it with evict_last priority
   TileRaster raster;
   int64_t tiles;
   int64_t tile_begin;     // first group-wide tile index of this problem

@@ -39,12 +39,12 @@ __device__ __forceinline__ bool pair_produce_tile(const GemmProblem& pr, const C
                                                   uint32_t bar_base, uint32_t leader_bar_base,
                                                   int& stage, uint32_t& phase, PipeCtl* ctl,
                                                   const GemmGroup& g, uint64_t pol_keep,
-                                                  uint64_t pol_stream, bool reverse_k) {
+                                                  uint64_t pol_normal, bool reverse_k) {
   const int am = mt * kPairBM + 128 * static_cast<int>(rank) + pr.a_mn_off;
   const int bm = nt * kBN + 128 * static_cast<int>(rank) + pr.b_mn_off;
   const int num_kb = pr.num_kb;
-  const uint64_t pol_a = pr.a_keep ? pol_keep : pol_stream;
-  const uint64_t pol_b = pr.a_keep ? pol_stream : pol_keep;
+  const uint64_t pol_a = pr.a_keep ? pol_keep : pol_normal;
+  const uint64_t pol_b = pr.b_keep ? pol_keep : pol_normal;
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_phase(bar_base + 8u * (kPairStages + stage), phase ^ 1u, ctl, g.err, g.timeout_ns))
       return false;
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return c >= g.total_tiles ? -1 : c;
       };
       const uint64_t pol_keep = l2_policy_evict_last();
-      const uint64_t pol_stream = l2_policy_evict_first();
+      const uint64_t pol_normal = l2_policy_evict_normal();
       int64_t claimed = rank == 0 ? claim() : -1;
       while (ok) {
         int64_t t;
@@ -240,16 +240,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p == 0)
           ok = pair_produce_tile<C0>(pr, &maps.a[0], &maps.b[0], mt, nt, rank, smem_base, bar_base,
                                      leader_bar_base, stage, phase, ctl, g, pol_keep,
-                                     pol_stream, rev);
+                                     pol_normal, rev);
         else if constexpr (C1::kValid) {
           if (p == 1)
             ok = pair_produce_tile<C1>(pr, &maps.a[1], &maps.b[1], mt, nt, rank, smem_base,
                                        bar_base, leader_bar_base, stage, phase, ctl, g,
-                                       pol_keep, pol_stream, rev);
+                                       pol_keep, pol_normal, rev);
           else if constexpr (C2::kValid)
             ok = pair_produce_tile<C2>(pr, &maps.a[2], &maps.b[2], mt, nt, rank, smem_base,
                                        bar_base, leader_bar_base, stage, phase, ctl, g,
-                                       pol_keep, pol_stream, rev);
+                                       pol_keep, pol_normal, rev);
         }
       }
       if (!ok) {
