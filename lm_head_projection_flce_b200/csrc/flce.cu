@@ -444,14 +444,45 @@ static bool tmap_mnmajor(CUtensorMap* tm, const void* base, int64_t mn, int64_t 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Raster that keeps operand panels resident in L2: when all of B (or all of A)
-// fits in the budget, iterate over its tiles fastest so it is read from HBM
-// once while the other operand streams; otherwise group m-tiles whose A panels
-// fit.
-constexpr int64_t kL2ResidentBytes = int64_t(40) << 20;
+// Tile order.  When all of one operand fits in L2 it is kept there (loaded
+// with evict_last) and the other streams from HBM once.  Otherwise tiles are
+// taken in groups of g rows (or columns) of tiles, the group's index running
+// fastest, and g and the orientation are chosen by a model of the HBM bytes
+// the operand panels cost:
+//   - the grouped operand is read once if the group's panels fit in L2 (and
+//     they are then kept with evict_last when the group lasts two waves or
+//     more, so later waves find them), else once per wave of the group;
+//   - the other operand is read once per group (its panel is shared by the
+//     group's g tiles, which run side by side), or once per wave when a wave
+//     spans several groups.
+// A wave is `pairs` tiles (the resident CTA pairs).
+constexpr int64_t kL2ResidentBytes = int64_t(40) << 20;  // a whole operand kept in L2
+constexpr int64_t kL2GroupBytes = int64_t(60) << 20;     // one group's panels kept in L2
 
-static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
-  TileRaster r{};
+struct RasterPlan {
+  TileRaster raster;
+  int a_keep, b_keep;
+};
+
+// Modelled HBM bytes of the operand panels for groups of g tiles along the
+// grouped operand (tiles_g of them, panel_g bytes each) against tiles_o tiles
+// of the other operand (panel_o bytes each).
+static double raster_bytes(int64_t tiles_g, int64_t tiles_o, double panel_g, double panel_o,
+                           int64_t g, double pairs, bool* keep) {
+  const double all_g = panel_g * double(tiles_g), all_o = panel_o * double(tiles_o);
+  const double waves_total = double(tiles_g) * double(tiles_o) / pairs;
+  const double waves_group = double(g) * double(tiles_o) / pairs;
+  const bool fits = double(g) * panel_g <= double(kL2GroupBytes);
+  *keep = fits && waves_group >= 2.0;
+  const double bytes_g = all_g * (fits ? 1.0 : std::max(1.0, waves_group));
+  const double groups = double(cdiv(tiles_g, g));
+  const double bytes_o = all_o * std::min(groups, std::max(1.0, waves_total));
+  return bytes_g + bytes_o;
+}
+
+static RasterPlan make_raster(int64_t m, int64_t n, int64_t k, int pairs) {
+  RasterPlan plan{};
+  TileRaster& r = plan.raster;
   r.m_tiles = int(cdiv(m, kTileRows));
   r.n_tiles = int(cdiv(n, kBN));
   const int64_t kk = std::max<int64_t>(k, 1);
@@ -460,17 +491,37 @@ static TileRaster make_raster(int64_t m, int64_t n, int64_t k) {
   if (a_all <= kL2ResidentBytes && a_all <= b_all) {
     r.n_fast = 0;
     r.group = r.m_tiles;
-  } else if (b_all <= kL2ResidentBytes) {
+    plan.a_keep = 1;
+    return plan;
+  }
+  if (b_all <= kL2ResidentBytes) {
     r.n_fast = 1;
     r.group = r.n_tiles;
-  } else {
-    r.n_fast = 0;
-    r.group = int(std::min<int64_t>(std::max<int64_t>(1, (int64_t(24) << 20) / a_panel), r.m_tiles));
+    plan.b_keep = 1;
+    return plan;
   }
-  return r;
+  const double p = double(std::max(pairs, 1));
+  double best = -1.0;
+  for (int fast = 0; fast < 2; ++fast) {
+    const int64_t tg = fast ? r.n_tiles : r.m_tiles, to = fast ? r.m_tiles : r.n_tiles;
+    const double pg = double(fast ? b_panel : a_panel), po = double(fast ? a_panel : b_panel);
+    for (int64_t g = 1; g <= tg; ++g) {
+      bool keep = false;
+      const double bytes = raster_bytes(tg, to, pg, po, g, p, &keep);
+      if (best < 0.0 || bytes < best * (1.0 - 1e-9)) {
+        best = bytes;
+        r.n_fast = fast;
+        r.group = int(g);
+        plan.a_keep = !fast && keep ? 1 : 0;
+        plan.b_keep = fast && keep ? 1 : 0;
+      }
+    }
+  }
+  return plan;
 }
 
-static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool b_mn, int epi) {
+static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool b_mn, int epi,
+                                int pairs) {
   GemmProblem p{};
   p.m = m;
   p.n = n;
@@ -479,12 +530,10 @@ static GemmProblem make_problem(int64_t m, int64_t n, int64_t k, bool a_mn, bool
   p.b_mn = b_mn;
   p.epi = epi;
   p.num_kb = int(cdiv(k, kBK));
-  p.raster = make_raster(m, n, k);
-  // Only an operand the raster holds whole in L2 (hidden, in the projection and
-  // recompute GEMMs and as dW's B) is worth protecting; a grouped panel of a
-  // larger operand is re-read only by tiles running at the same time.
-  p.a_keep = !p.raster.n_fast && p.raster.group == p.raster.m_tiles ? 1 : 0;
-  p.b_keep = p.raster.n_fast && p.raster.group == p.raster.n_tiles ? 1 : 0;
+  const RasterPlan rp = make_raster(m, n, k, pairs);
+  p.raster = rp.raster;
+  p.a_keep = rp.a_keep;
+  p.b_keep = rp.b_keep;
   p.tiles = (m > 0 && n > 0) ? int64_t(p.raster.m_tiles) * p.raster.n_tiles : 0;
   return p;
 }
@@ -621,7 +670,7 @@ static FwdPlan plan_forward(const Shape& s) {
 }
 
 static int64_t default_chunk(const Shape& s) {
-  const int64_t cap = cdiv(cdiv(s.v, 6), kBN) * kBN;  // at most a sixth of the vocabulary
+  const int64_t cap = cdiv(cdiv(s.v, 5), kBN) * kBN;  // at most a fifth of the vocabulary
   int64_t budget = int64_t(kChunkBudgetBytes / (2 * size_t(std::max<int64_t>(s.n, 1))));
   budget = budget / kBN * kBN;
   return std::max<int64_t>(kBN, std::min(cap, std::max(kMinChunk, budget)));
@@ -753,7 +802,7 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   CUtensorMap ta, tb;
   if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBBoxRows))
     return FLCE_ERR_CUDA;
-  const GemmProblem prob = make_problem(n, v, h, false, false, kEpiForward);
+  const GemmProblem prob = make_problem(n, v, h, false, false, kEpiForward, dev->num_sms / 2);
   EpiSet<kEpiSetForward> es{};
   EpiForward::Params& ep = es.fwd;
   ep.labels = labels;
@@ -877,7 +926,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   // K3 for chunk c: problem, maps and epilogue parameters.
   auto grad_problem = [&](int64_t c, GemmProblem* pr, CUtensorMap* ma, CUtensorMap* mb,
                           EpiGrad::Params* ep) {
-    *pr = make_problem(n, chunk_width(c), h, false, false, kEpiGrad);
+    *pr = make_problem(n, chunk_width(c), h, false, false, kEpiGrad, dev->num_sms / 2);
     pr->b_mn_off = int(chunk_v0(c));
     *ma = t_hid_k;
     *mb = t_w_k;
@@ -920,7 +969,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     int count = 0;
     double flops = 0.0, bytes = 0.0;
     // K5: dhidden (+)= G . W[v0 : v0 + width]  (contraction over the chunk; long tiles first)
-    pr[count] = make_problem(n, h, gcols, false, true, kEpiAccumRows);
+    pr[count] = make_problem(n, h, gcols, false, true, kEpiAccumRows, dev->num_sms / 2);
     pr[count].b_k_off = int(v0);
     ma[count] = t_g_k;
     mb[count] = t_w_mn;
@@ -937,7 +986,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     }
     ++count;
     // K4: dW[v0 : v0 + width] = G^T . hidden  (contraction over tokens)
-    pr[count] = make_problem(width, h, n, true, true, kEpiStoreRows);
+    pr[count] = make_problem(width, h, n, true, true, kEpiStoreRows, dev->num_sms / 2);
     ma[count] = t_g_mn;
     mb[count] = t_hid_mn;
     es.store.out = static_cast<uint8_t*>(dweight) + size_t(v0) * h * wsz;
@@ -1006,7 +1055,8 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   const bool ok_a = a_mn ? tmap_mnmajor(&ta, a, m, k, m) : tmap_kmajor(&ta, a, k, m, k, kBM);
   const bool ok_b = b_mn ? tmap_mnmajor(&tb, b, n, k, n) : tmap_kmajor(&tb, b, k, n, k, kBBoxRows);
   if (!ok_a || !ok_b) return FLCE_ERR_CUDA;
-  const GemmProblem prob = make_problem(m, n, k, a_mn != 0, b_mn != 0, kEpiStoreRows);
+  const GemmProblem prob = make_problem(m, n, k, a_mn != 0, b_mn != 0, kEpiStoreRows,
+                                        dev->num_sms / 2);
   EpiSet<kEpiSetStore> es{};
   EpiStoreRows::Params& ep = es.store;
   ep.out = d;

@@ -4,7 +4,7 @@
 //
 // CTA r of the pair loads A rows [128 r, 128 r + 128) and B rows
 // [128 r, 128 r + 128) of the tile into its own shared memory (32 KB per
-// 64-deep k-block, 6 stages) and receives D rows [128 r, 128 r + 128) in its
+// 64-deep k-block, 7 stages: 224 KB) and receives D rows [128 r, 128 r + 128) in its
 // own tensor memory.  Per SM this moves two thirds of the operand bytes of a
 // 128 x 256 single-CTA tile for the same FLOPs.
 //
@@ -25,7 +25,7 @@
 namespace flce {
 
 constexpr int kPairBM = 256;  // rows of a pair tile (128 per CTA)
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 7;
 constexpr uint32_t kPairATileBytes = 128 * kBK * 2;  // this CTA's 128 A rows x 64 K
 constexpr uint32_t kPairBTileBytes = 128 * kBK * 2;  // this CTA's 128 of B's 256 rows x 64 K
 constexpr uint32_t kPairStageBytes = kPairATileBytes + kPairBTileBytes;  // 32 KB
