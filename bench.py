@@ -114,12 +114,19 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "timestamp")
 
     def __init__(self, gpu_uuid: str | None):
         self.proc = None
         self.path = None
         self.uuid = gpu_uuid
+        self.window = None
+
+    def mark(self, begin: float, end: float):
+        """Host wall-clock bounds of the timed region: only samples taken inside it
+        (plus one sampling period after it) are summarised."""
+        self.window = (begin, end + 0.1)
 
     def start(self):
         fd, self.path = tempfile.mkstemp(prefix="flce_clocks_", suffix=".csv")
@@ -146,11 +153,29 @@ class ClockSampler:
             rows = open(self.path).read().splitlines()
         finally:
             os.unlink(self.path)
-        return self.summarize(rows)
+        return self.summarize(rows, self.window)
 
     @staticmethod
-    def summarize(rows: list[str]) -> dict:
-        """Median SM clock, max clock and the throttle reasons seen in the CSV rows."""
+    def sample_time(field: str) -> float | None:
+        """nvidia-smi's timestamp (local time, 'YYYY/MM/DD HH:MM:SS.mmm') as epoch seconds."""
+        try:
+            return datetime.datetime.strptime(field.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    @staticmethod
+    def summarize(rows: list[str], window: tuple | None = None) -> dict:
+        """Median SM clock, max clock and the throttle reasons seen in the CSV rows
+        (only rows whose timestamp lies in `window`, when one is given and some do)."""
+        if window is not None:
+            inside = []
+            for row in rows:
+                c = [x.strip() for x in row.split(",")]
+                t = ClockSampler.sample_time(c[9]) if len(c) >= 10 else None
+                if t is not None and window[0] <= t <= window[1]:
+                    inside.append(row)
+            if inside:
+                rows = inside
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for row in rows:
@@ -415,11 +440,13 @@ class Timer:
             flce.profile_start()
         l0 = flce.launch_count()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        t_begin = time.time()
         ev[0].record(self.stream)
         for k in range(steps):
             step()
             ev[k + 1].record(self.stream)
         torch.cuda.synchronize(self.dev)
+        sampler.mark(t_begin, time.time())
         self.barrier()
         launches = flce.launch_count() - l0
         stats = flce.profile_stop() if profile else {}

@@ -99,6 +99,20 @@ def test_clock_summary():
     assert "hw_slowdown" in bad["reasons"] and bench.BAD_REASONS & set(bad["reasons"])
 
 
+def test_clock_summary_keeps_the_timed_window():
+    row = "0, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, {cap}, 2026/12/03 07:26:{sec}"
+    rows = [row.format(mhz=1965, cap="Not Active", sec="54.100"),      # idle, before the region
+            row.format(mhz=1965, cap="Not Active", sec="54.200"),
+            row.format(mhz=1290, cap="Active", sec="54.300"),          # under load
+            row.format(mhz=1275, cap="Active", sec="54.400")]
+    t = bench.ClockSampler.sample_time("2026/12/03 07:26:54.250")
+    c = bench.ClockSampler.summarize(rows, (t, t + 0.2))
+    assert c["samples"] == 2 and c["sm_mhz"] == 1282.5 and c["reasons"] == ["sw_power_cap"]
+    # no sample inside the window: all rows are used rather than none
+    assert bench.ClockSampler.summarize(rows, (t + 10, t + 11))["samples"] == 4
+    assert bench.ClockSampler.summarize(rows)["samples"] == 4
+
+
 def test_committed_traffic_needs_matching_sources(tmp_path, monkeypatch):
     f = tmp_path / "t.json"
     dig = bench.kernel_source_digest()
