@@ -276,12 +276,15 @@ def cpu_baseline(w, d, target_s: float = 15.0, max_tokens: int = 4096) -> dict:
         if dt >= target_s / 4 or s >= min(max_tokens, w.n_tokens):
             break
         s = min(4 * s, max_tokens, w.n_tokens)
-    # The timed sample: scaled so that one oracle pass takes about target_s.
-    s = int(min(max_tokens, w.n_tokens, max(s, s * target_s / max(dt, 1e-3))))
-    rows = rng.choice(w.n_tokens, size=s, replace=False)
-    t0 = time.perf_counter()
-    oracle_step(O, w, hidden, weight, labels, rows, nlt)
-    dt = time.perf_counter() - t0
+    # The timed sample: scaled so that one oracle pass takes about target_s (the
+    # last probe already is that pass when the size does not change).
+    s_next = int(min(max_tokens, w.n_tokens, max(s, s * target_s / max(dt, 1e-3))))
+    if s_next != s:
+        s = s_next
+        rows = rng.choice(w.n_tokens, size=s, replace=False)
+        t0 = time.perf_counter()
+        oracle_step(O, w, hidden, weight, labels, rows, nlt)
+        dt = time.perf_counter() - t0
     return {"value": s / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": (f"{s} seeded tokens of {w.name} through the FP64 oracle's full forward + "
                        f"backward (lse over all {w.vocab} rows, their dhidden rows and their "
