@@ -596,13 +596,18 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kPairSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // Programmatic dependent launch: the kernel's set-up may overlap the tail of
+  // the previous kernel in the stream; it waits (griddepcontrol.wait) before
+  // reading or writing anything else.
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   LaunchScope scope(family, flops, bytes, st);
   if (cudaLaunchKernelEx(&cfg, kern, maps, g, ep) != cudaSuccess) return FLCE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;

@@ -167,6 +167,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after_sync();
+  // The set-up above (barriers, tensor-map prefetch, TMEM) touches nothing the
+  // previous launch writes, so with a programmatic dependent launch it overlaps
+  // that launch's tail; everything below may read its results.  The next launch
+  // may be scheduled right away: its CTAs take SMs as ours exit and wait too.
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
   const int64_t pair_id = blockIdx.x >> 1;
   const int64_t num_pairs = gridDim.x >> 1;

@@ -88,6 +88,18 @@ __host__ __device__ constexpr uint32_t mma_idesc_bf16(int m, int n, bool a_mn_ma
          | (static_cast<uint32_t>(m >> 4) << 24);     // M / 16
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Block until the grids this one depends on (stream order) have completed and
+// their memory is visible; a no-op when the launch did not allow overlap.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the next launch in the stream be scheduled (it still waits for this
+// grid's completion before touching memory, through grid_dependency_wait).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
