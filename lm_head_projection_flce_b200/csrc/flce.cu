@@ -53,7 +53,7 @@ __device__ unsigned int g_device_error;  // per-device sticky error word (kDevEr
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr int kMergeRows = 32;                         // token rows per merge block
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 16;
 constexpr int kFinalThreads = 256;
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1024;  // TMA coordinates are int32
 constexpr size_t kAlign = 1024;
@@ -87,7 +87,7 @@ __global__ void zero16_kernel(uint4* __restrict__ dst, int64_t n16) {
     dst[i] = make_uint4(0, 0, 0, 0);
 }
 
-// K2: merge the per-tile partials of 32 token rows (8 warps split the tiles),
+// K2: merge the per-tile partials of 32 token rows (16 warps split the tiles),
 // then per token: lse, token loss, label check (mask: optional, 0 = ignore the
 // token); per block: loss and count sums.  Also finishes the cross entropy on
 // given logits, whose row segments leave partials in the same layout.
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kMergeRows* kMergeWarps)
   const int64_t n = int64_t(blockIdx.x) * kMergeRows + lane;
   float M = -INFINITY, S = 0.0f;
   if (n < n_tokens) {
+#pragma unroll 4
     for (int t = warp; t < v_tiles; t += kMergeWarps) {
       const float m = part_m[int64_t(t) * n_tokens + n];
       const float s = part_s[int64_t(t) * n_tokens + n];
