@@ -308,7 +308,13 @@ class _FusedLinearCE(torch.autograd.Function):
 def fused_linear_cross_entropy(hidden, weight, labels, *, ignore_index: int = -100,
                                softcap: float = 0.0, unpadded_vocab: int | None = None,
                                reduction: str = "sum", num_label_tokens: int | None = None):
-    """Autograd-aware loss: gradients flow to ``hidden`` and ``weight``."""
+    """Autograd-aware loss: gradients flow to ``hidden`` and ``weight``.
+
+    With an FP32 head the forward's workspace (which holds the head's BF16
+    copy, V x H x 2 bytes, and the backward's buffers) is kept until the
+    backward runs, so the head is cast once per step; a BF16 head keeps
+    nothing between the two.
+    """
     return _FusedLinearCE.apply(hidden, weight, labels, ignore_index, softcap, unpadded_vocab,
                                 reduction, num_label_tokens)
 
