@@ -18,7 +18,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(port, out):
+def _worker(port, out, head_dtype="bf16"):
     import sys
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -34,7 +34,8 @@ def _worker(port, out):
     torch.cuda.set_device(dev)
     dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev)
     try:
-        w = W.custom(700, 520, 5000, 5120, softcap=30.0, ignore_frac=0.1, w_sigma=0.05, seed=41)
+        w = W.custom(700, 520, 5000, 5120, softcap=30.0, ignore_frac=0.1, w_sigma=0.05, seed=41,
+                     w_dtype=head_dtype)
         d = W.generate(w)
         hid = d["hidden"].to(dev).requires_grad_(True)
         lab = d["labels"].to(dev)
@@ -58,12 +59,16 @@ def _worker(port, out):
         dist.destroy_process_group()
 
 
-def test_data_parallel_wrapper_single_rank_nccl():
+@pytest.mark.parametrize("head_dtype", ["bf16", "f32"])
+def test_data_parallel_wrapper_single_rank_nccl(head_dtype):
+    """The wrapper over a one-rank group equals the plain fused loss bit for bit,
+    for a BF16 head and for FP32 master weights (whose BF16 copy the autograd
+    wrapper keeps from the forward for the backward)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    p = ctx.Process(target=_worker, args=(_free_port(), q))
+    p = ctx.Process(target=_worker, args=(_free_port(), q, head_dtype))
     p.start()
     p.join(timeout=300)
     assert p.exitcode == 0
