@@ -50,6 +50,11 @@ CASES = {
     "ktail_softcap_padded": W.custom(700, 520, 5000, 5120, softcap=30.0, ignore_frac=0.1,
                                      w_sigma=0.05, seed=13),
     "zipf_labels": W.custom(512, 256, 3000, 3000, label_dist="zipf", ignore_frac=0.2, seed=14),
+    # hidden (12 ragged 256-row tiles x 8200 = 49 MB) is too large to stay in L2 whole, so the
+    # projection and recompute GEMMs take their tile order from the traffic model; ragged
+    # edges in every dimension (3000 tokens, 8200 = 128 x 64 + 8 hidden, 20011 of 20480 rows)
+    "fallback_raster_ragged": W.custom(3000, 8200, 20011, 20480, softcap=30.0, ignore_frac=0.05,
+                                       w_sigma=0.01, seed=15),
 }
 
 
