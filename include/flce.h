@@ -34,9 +34,10 @@
  *    undefined.
  *  - After one call of an entry point per device and dtype (which queries the
  *    device, resolves the tensor-map encoder and caches launch shapes),
- *    flce_forward / flce_backward / flce_ce_* only enqueue kernels on
- *    `stream`, so a sequence of them can be captured into a CUDA graph and
- *    replayed with the same buffers.
+ *    flce_forward / flce_backward / flce_ce_* only enqueue work on `stream`
+ *    (kernels, and in flce_forward one 4-byte memset that zeroes a tile
+ *    counter in the workspace), so a sequence of them can be captured into a
+ *    CUDA graph and replayed with the same buffers.
  *  - Labels outside [0, V) that are not ignore_index cannot be checked on the
  *    host without a device read; the kernels treat them as ignored (zero loss,
  *    zero gradient) and raise FLCE_ERR_BAD_LABEL in a per-device error word

@@ -269,9 +269,13 @@ static DeviceInfo g_dev[64];
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // Id of the calling thread's current CUDA context, 0 when it has none (for
-// instance right after cudaDeviceReset, until the runtime creates a new one).
-// Device addresses looked up in one context (the error word, the no-allocation
-// scratch array) are stale in the next, so they are cached with this id.
+// instance right after cudaDeviceReset, until the runtime creates a new one),
+// kContextUnknown when the driver cannot tell.  Device addresses looked up in
+// one context (the error word, the no-allocation scratch array) are stale in
+// the next, so they are cached with this id and looked up again when it
+// changes; with kContextUnknown the cache is kept.
+constexpr unsigned long long kContextUnknown = ~0ull;
+
 static unsigned long long current_context_id() {
   static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
   static PFN_cuCtxGetId_v12000 get_id = nullptr;
@@ -287,12 +291,18 @@ static unsigned long long current_context_id() {
         q == cudaDriverEntryPointSuccess)
       get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
   });
-  if (get_current == nullptr || get_id == nullptr) return 0;
+  if (get_current == nullptr || get_id == nullptr) return kContextUnknown;
   CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return kContextUnknown;
+  if (ctx == nullptr) return 0;
   unsigned long long id = 0;
-  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
-    return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return kContextUnknown;
   return id;
+}
+
+// True when addresses cached in context `cached` must be looked up again.
+static bool context_changed(unsigned long long now, unsigned long long cached) {
+  return now != kContextUnknown && (now == 0 || now != cached);
 }
 
 static int device_info(DeviceInfo** out) {
@@ -301,7 +311,7 @@ static int device_info(DeviceInfo** out) {
   const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& d = g_dev[dev];
-  if (d.init && (ctx == 0 || ctx != d.ctx_id)) d.init = false;  // a new context: look up again
+  if (d.init && context_changed(ctx, d.ctx_id)) d.init = false;  // a new context: look up again
   if (!d.init) {
     d.init = true;
     d.status = FLCE_OK;
@@ -1194,7 +1204,7 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
     // the kernels get this looked-up pointer instead.
     const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_addr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
+    if (g_noalloc_addr[dev] == nullptr || context_changed(ctx, g_noalloc_ctx[dev])) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
         return FLCE_ERR_CUDA;
