@@ -486,6 +486,8 @@ class FlceRun:
         self.kw = dict(softcap=w.softcap, unpadded_vocab=v, reduction=w.reduction,
                        num_label_tokens=self.nlt, workspace=self.ws)
         self.reuse = self.wt.dtype == torch.float32
+        self.fused_cast = False
+        self.label = w.name  # names the committed traffic record this run's kernels match
         self.captured = None
         self.graph_launches = 0
         if graph:
@@ -496,6 +498,21 @@ class FlceRun:
             self.graph_launches = (flce.launch_count() - l0) // 2  # eager set-up + capture
             self.loss = self.captured.loss
 
+    def use_fused_head_cast(self, dev):
+        """Switch an FP32-head run to FLCE_FUSED_HEAD_CAST: the GEMMs round the
+        head in the kernel, with the smaller workspace that has no BF16 copy."""
+        import torch
+        from lm_head_projection_flce_b200 import flce
+        w = self.w
+        self.ws = None
+        self.ws = torch.empty(flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab,
+                                                  self.wt.dtype, fused_head_cast=True),
+                              dtype=torch.uint8, device=dev)
+        self.kw["workspace"] = self.ws
+        self.reuse = False
+        self.fused_cast = True
+        self.label = w.name + "/fused_head_cast"
+
     def step(self, h_in=None, l_in=None):
         from lm_head_projection_flce_b200 import flce
         if self.captured is not None:
@@ -505,9 +522,10 @@ class FlceRun:
             return
         h_in = self.hid if h_in is None else h_in
         l_in = self.lab if l_in is None else l_in
-        flce.forward(h_in, self.wt, l_in, loss=self.loss, lse=self.lse, **self.kw)
+        flce.forward(h_in, self.wt, l_in, loss=self.loss, lse=self.lse,
+                     fused_head_cast=self.fused_cast, **self.kw)
         flce.backward(h_in, self.wt, l_in, self.lse, self.grad, dhidden=self.dh, dweight=self.dw,
-                      reuse_head_copy=self.reuse, **self.kw)
+                      reuse_head_copy=self.reuse, fused_head_cast=self.fused_cast, **self.kw)
 
 
 def measure_flce(run: "FlceRun", timer: "Timer", steps: int, warmup: int, world: int,
@@ -540,14 +558,14 @@ def measure_flce(run: "FlceRun", timer: "Timer", steps: int, warmup: int, world:
     w = run.w
     path_flops = w.flops_fwd_bwd * steps
     if prof is not None:
-        roof = tensor_roofline(prof["stats"], peaks, peak_src, w.name, path_flops, ms_max)
+        roof = tensor_roofline(prof["stats"], peaks, peak_src, run.label, path_flops, ms_max)
         kernels = kernel_table(prof["stats"], steps)
         launches = head["launches"]
     else:  # graph replays carry no per-launch events: the whole step is the unit
         stats = {"whole step (CUDA graph replay)": {
             "flops": path_flops, "total_ms": ms_max, "launches": run.graph_launches * steps,
             "bytes": 0.0}}
-        roof = tensor_roofline(stats, peaks, peak_src, w.name, path_flops, ms_max)
+        roof = tensor_roofline(stats, peaks, peak_src, run.label, path_flops, ms_max)
         kernels = {}
         launches = run.graph_launches * steps
     return {"ms": ms_max, "per_step": head["per_step"], "launches": launches,
@@ -690,16 +708,26 @@ def run_ours(args, w) -> int:
                 continue
             rx = FlceRun(wx, dev)
             k = max(5, args.extra_steps)
+
+            def extra_entry(mx, config):
+                return {"value": wx.n_tokens * k / (mx["ms"] / 1e3), "unit": UNIT, "steps": k,
+                        "warmup": 3, "ms_per_step": mx["ms"] / k,
+                        "ms_per_step_median": statistics.median(mx["per_step"]),
+                        "config": config, "roofline": mx["roofline"], "kernels": mx["kernels"],
+                        "gpu_launches": mx["launches"], "clocks": mx["clocks"]}
+
             mx = measure_flce(rx, timer, k, 3, 1, lambda x: x, peaks, peak_src)
-            entry = {"value": wx.n_tokens * k / (mx["ms"] / 1e3), "unit": UNIT, "steps": k,
-                     "warmup": 3, "ms_per_step": mx["ms"] / k,
-                     "ms_per_step_median": statistics.median(mx["per_step"]),
-                     "config": workload_config(wx, "one GPU"), "roofline": mx["roofline"],
-                     "kernels": mx["kernels"], "gpu_launches": mx["launches"],
-                     "clocks": mx["clocks"]}
+            entry = extra_entry(mx, workload_config(wx, "one GPU"))
             if not args.no_cpu_baseline:
                 entry["cpu_baseline"] = cpu_baseline(wx, rx.data, target_s=6.0)
             extras[wx.name] = entry
+            if wx.w_dtype == "f32":
+                # the same workload with the head rounded inside the GEMMs (no BF16 copy)
+                rx.use_fused_head_cast(dev)
+                mx = measure_flce(rx, timer, k, 3, 1, lambda x: x, peaks, peak_src)
+                cfg = {**workload_config(wx, "one GPU"), "head_cast": "fused into the GEMMs",
+                       "workspace_bytes": int(rx.ws.numel())}
+                extras[wx.name + "/fused_head_cast"] = extra_entry(mx, cfg)
             del rx
             torch.cuda.empty_cache()
         extras[W.CE_LOGITS.name] = measure_chunked_ce(

@@ -81,6 +81,26 @@ size_t flce_workspace_min_size(int64_t n_tokens, int64_t hidden, int64_t padded_
                                int64_t unpadded_vocab, int w_dtype);
 
 /*
+ * FP32 head without a BF16 copy (inkling2 page, Inkling2FusedLinearCrossEntropy
+ * class docstring: an FP32 head is rounded to BF16, "the cast FSDP applies").
+ * With this flag, flce_forward_ex and flce_backward_ex do not write the
+ * head's BF16 copy (V*H*2 bytes) into the workspace: the GEMMs that read the
+ * head load its FP32 rows and round them to BF16 (nearest even, the same
+ * rounding as the copy) in shared memory, inside the kernel.  Results are
+ * bit-identical to the copy's; the workspace shrinks by the copy, and the
+ * GEMMs move twice the head bytes and convert every head tile once per tile
+ * row, so they run slower than the copy path (measured in the design notes).
+ * The flag has no effect with a BF16 head.
+ * The _ex sizes take the same flags (0 or FLCE_FUSED_HEAD_CAST; any other
+ * bit gives 0).
+ */
+#define FLCE_FUSED_HEAD_CAST 2u
+size_t flce_workspace_size_ex(int64_t n_tokens, int64_t hidden, int64_t padded_vocab,
+                              int64_t unpadded_vocab, int w_dtype, unsigned int flags);
+size_t flce_workspace_min_size_ex(int64_t n_tokens, int64_t hidden, int64_t padded_vocab,
+                                  int64_t unpadded_vocab, int w_dtype, unsigned int flags);
+
+/*
  * Forward: the loss and the per-token logsumexp.
  *   Defines: linear_ce page, FusedLinearCrossEntropy(ignore_index=-100,
  *   logit_softcapping=0, reduction='sum') and forward(hidden_states, labels,
@@ -105,6 +125,19 @@ int flce_forward(const void* hidden, const void* weight, int w_dtype, const int6
                  int64_t unpadded_vocab, int64_t ignore_index, float softcap,
                  int reduction, int64_t num_label_tokens, float* loss, float* lse,
                  void* workspace, size_t ws_bytes, flce_stream_t stream);
+
+/*
+ * flce_forward with option flags: 0 or FLCE_FUSED_HEAD_CAST (see above; the
+ * workspace then needs flce_workspace_size_ex(..., FLCE_FUSED_HEAD_CAST)
+ * bytes).  Any other bit set: FLCE_ERR_INVALID_ARG.
+ * flce_forward(...) is flce_forward_ex(..., 0, stream).
+ */
+int flce_forward_ex(const void* hidden, const void* weight, int w_dtype,
+                    const int64_t* labels, int64_t n_tokens, int64_t hidden_size,
+                    int64_t padded_vocab, int64_t unpadded_vocab, int64_t ignore_index,
+                    float softcap, int reduction, int64_t num_label_tokens, float* loss,
+                    float* lse, void* workspace, size_t ws_bytes, unsigned int flags,
+                    flce_stream_t stream);
 
 /*
  * Backward: gradients of the loss above, recomputing the logits.
@@ -143,7 +176,11 @@ int flce_backward(const void* hidden, const void* weight, int w_dtype, const int
  *          of V*H*4 bytes and one write of V*H*2).  The flag is ignored for a
  *          BF16 head, which is used in place.  The library cannot check the
  *          promise: a stale copy gives wrong gradients without an error.
- *          Any other bit set: FLCE_ERR_INVALID_ARG.
+ *          Or FLCE_FUSED_HEAD_CAST: no copy is used or written; the recompute
+ *          and dhidden GEMMs round the FP32 head in the kernel (the workspace
+ *          then needs flce_workspace_min_size_ex(..., FLCE_FUSED_HEAD_CAST)
+ *          bytes at least).  Both flags at once, or any other bit set:
+ *          FLCE_ERR_INVALID_ARG.
  * flce_backward(...) is flce_backward_ex(..., 0, stream).
  */
 #define FLCE_BWD_HEAD_COPY_VALID 1u
@@ -230,9 +267,10 @@ int flce_ce_backward(const void* logits, int dtype, const int64_t* labels, const
  *   Scratch: a 32 MiB array in this library's device memory, present on every
  *   GPU that loads the library until the process exits.  A problem whose
  *   forward scratch (8 B x ceil(V/256) x N for the logsumexp partials, plus
- *   4 B x N, plus the BF16 copy of an FP32 head) exceeds 32 MiB is refused
- *   with FLCE_ERR_WORKSPACE and nothing is enqueued; e.g. N = 4096 tokens with
- *   V = 128256 and a BF16 head needs 15.7 MiB (16.4 MB) and fits.
+ *   4 B x N) exceeds 32 MiB is refused with FLCE_ERR_WORKSPACE and nothing is
+ *   enqueued; e.g. N = 4096 tokens with V = 128256 needs 15.7 MiB (16.4 MB)
+ *   and fits.  An FP32 head takes the FLCE_FUSED_HEAD_CAST path (rounded to
+ *   BF16 inside the GEMM), so it needs no room for a BF16 copy.
  *   The array is shared by every call on a device and keeps whatever the last
  *   call left in it; the forward writes every scratch byte before reading it,
  *   so nothing has to be cleared between calls.  Calls that overlap on the GPU

@@ -426,14 +426,17 @@ class LaunchScope {
   bool active_ = false;
 };
 
-// 2-D BF16 tensor map, 128-byte swizzle, zero fill outside [inner, outer).
+// 2-D BF16 (or FP32) tensor map, 128-byte swizzle, zero fill outside [inner, outer).
 static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
-                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                      bool f32 = false) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+  const CUresult r = g_encode(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                              2, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -450,6 +453,17 @@ static bool tmap_kmajor(CUtensorMap* tm, const void* base, int64_t k, int64_t ro
 static bool tmap_mnmajor(CUtensorMap* tm, const void* base, int64_t mn, int64_t k,
                          int64_t ld_elems) {
   return make_tmap(tm, base, uint64_t(mn), uint64_t(k), uint64_t(ld_elems) * 2, 64, 64);
+}
+// FP32 B operands for the in-kernel conversion (128-byte rows of 32 values):
+// K-major [rows][K] as boxes of 32 K x 128 rows, MN-major [K rows][MN] as boxes
+// of 32 MN x 64 K rows.
+static bool tmap_kmajor_f32(CUtensorMap* tm, const void* base, int64_t k, int64_t rows,
+                            int64_t ld_elems) {
+  return make_tmap(tm, base, uint64_t(k), uint64_t(rows), uint64_t(ld_elems) * 4, 32, 128, true);
+}
+static bool tmap_mnmajor_f32(CUtensorMap* tm, const void* base, int64_t mn, int64_t k,
+                             int64_t ld_elems) {
+  return make_tmap(tm, base, uint64_t(mn), uint64_t(k), uint64_t(ld_elems) * 4, 32, 64, true);
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -575,18 +589,20 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   g.tile_counter = counter;
   g.err = dev.err;
   g.timeout_ns = kDefaultTimeoutNs;
+  using Layout = PairLayoutOf<C0, C1, C2>;
   auto kern = tc_gemm_pair_kernel<EpiSet<kKinds>, C0, C1, C2>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(kPairSmemBytes)) != cudaSuccess)
+                           int(Layout::kSmemBytes)) != cudaSuccess)
     return FLCE_ERR_CUDA;
   // Pairs that can be resident at once (clusters need two SMs of one GPC);
-  // queried once per device (every instantiation shares the launch shape).
+  // queried once per device: every instantiation takes the same shared memory,
+  // which limits it to one CTA per SM whatever its thread count.
   int max_pairs = dev.max_pairs;
   if (max_pairs == 0) {
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2 * (dev.num_sms / 2), 1, 1);
-    q.blockDim = dim3(kThreads, 1, 1);
-    q.dynamicSmemBytes = kPairSmemBytes;
+    q.blockDim = dim3(Layout::kBlockThreads, 1, 1);
+    q.dynamicSmemBytes = Layout::kSmemBytes;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
     qa[0].val.clusterDim.x = 2;
@@ -604,8 +620,8 @@ static int launch_group(const GemmProblem* probs, const CUtensorMap* maps_a,
   const int pairs = int(std::min<int64_t>(max_pairs, total));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.blockDim = dim3(Layout::kBlockThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -649,6 +665,7 @@ static int launch_cast(const float* src, __nv_bfloat16* dst, int64_t elems,
 struct Shape {
   int64_t n, h, vp, v;
   int w_dtype;
+  int fused_cast;  // 1: an FP32 head is rounded inside the GEMMs; no BF16 copy
 };
 
 struct FwdPlan {
@@ -666,7 +683,7 @@ struct BwdPlan {
 // given the forward's workspace finds the copy the forward wrote there
 // (flce_backward_ex with FLCE_BWD_HEAD_COPY_VALID).
 static size_t head_copy_bytes(const Shape& s) {
-  return s.w_dtype == FLCE_F32 ? align_up(size_t(s.v) * s.h * 2) : 0;
+  return s.w_dtype == FLCE_F32 && !s.fused_cast ? align_up(size_t(s.v) * s.h * 2) : 0;
 }
 
 static FwdPlan plan_forward(const Shape& s) {
@@ -741,20 +758,30 @@ using namespace flce;
 
 // ====================================================================== C ABI
 
+extern "C" size_t flce_workspace_size_ex(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
+                                         int w_dtype, unsigned int flags) {
+  const int64_t v = unpadded <= 0 ? vp : unpadded;
+  if (!shape_ok(n, h, vp, v, w_dtype) || (flags & ~FLCE_FUSED_HEAD_CAST) != 0u) return 0;
+  const Shape s{n, h, vp, v, w_dtype, (flags & FLCE_FUSED_HEAD_CAST) ? 1 : 0};
+  return std::max(plan_forward(s).total, plan_backward(s, default_chunk(s)).total);
+}
+
 extern "C" size_t flce_workspace_size(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
                                       int w_dtype) {
+  return flce_workspace_size_ex(n, h, vp, unpadded, w_dtype, 0u);
+}
+
+extern "C" size_t flce_workspace_min_size_ex(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
+                                             int w_dtype, unsigned int flags) {
   const int64_t v = unpadded <= 0 ? vp : unpadded;
-  if (!shape_ok(n, h, vp, v, w_dtype)) return 0;
-  const Shape s{n, h, vp, v, w_dtype};
-  return std::max(plan_forward(s).total, plan_backward(s, default_chunk(s)).total);
+  if (!shape_ok(n, h, vp, v, w_dtype) || (flags & ~FLCE_FUSED_HEAD_CAST) != 0u) return 0;
+  const Shape s{n, h, vp, v, w_dtype, (flags & FLCE_FUSED_HEAD_CAST) ? 1 : 0};
+  return std::max(plan_forward(s).total, plan_backward(s, kBN).total);
 }
 
 extern "C" size_t flce_workspace_min_size(int64_t n, int64_t h, int64_t vp, int64_t unpadded,
                                           int w_dtype) {
-  const int64_t v = unpadded <= 0 ? vp : unpadded;
-  if (!shape_ok(n, h, vp, v, w_dtype)) return 0;
-  const Shape s{n, h, vp, v, w_dtype};
-  return std::max(plan_forward(s).total, plan_backward(s, kBN).total);
+  return flce_workspace_min_size_ex(n, h, vp, unpadded, w_dtype, 0u);
 }
 
 extern "C" double flce_flops_fwd_bwd(int64_t n, int64_t h, int64_t v) {
@@ -774,20 +801,23 @@ extern "C" const char* flce_status_string(int status) {
   }
 }
 
-extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
-                            const int64_t* labels, int64_t n, int64_t h, int64_t vp,
-                            int64_t unpadded, int64_t ignore_index, float softcap, int reduction,
-                            int64_t num_label_tokens, float* loss, float* lse, void* workspace,
-                            size_t ws_bytes, flce_stream_t stream) {
+extern "C" int flce_forward_ex(const void* hidden, const void* weight, int w_dtype,
+                               const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                               int64_t unpadded, int64_t ignore_index, float softcap,
+                               int reduction, int64_t num_label_tokens, float* loss, float* lse,
+                               void* workspace, size_t ws_bytes, unsigned int flags,
+                               flce_stream_t stream) {
   NvtxRange range("flce_forward");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
+  if ((flags & ~FLCE_FUSED_HEAD_CAST) != 0u) return FLCE_ERR_INVALID_ARG;
+  const bool fused = (flags & FLCE_FUSED_HEAD_CAST) != 0u && w_dtype == FLCE_F32;
   int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
                         num_label_tokens);
   if (st != FLCE_OK) return st;
   if ((n > 0 || reduction != FLCE_NONE) && (loss == nullptr || !aligned(loss, 4)))
     return FLCE_ERR_INVALID_ARG;
   if (n > 0 && (lse == nullptr || !aligned(lse, 4))) return FLCE_ERR_INVALID_ARG;
-  const Shape s{n, h, vp, v, w_dtype};
+  const Shape s{n, h, vp, v, w_dtype, fused ? 1 : 0};
   const FwdPlan p = plan_forward(s);
   if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p.total)
     return FLCE_ERR_WORKSPACE;
@@ -807,7 +837,7 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   }
 
   const void* wb = weight;
-  if (w_dtype == FLCE_F32) {
+  if (w_dtype == FLCE_F32 && !fused) {
     wb = ws + p.off_wb;
     if ((st = launch_cast(static_cast<const float*>(weight),
                           reinterpret_cast<__nv_bfloat16*>(ws + p.off_wb), v * h, *dev, cs)) !=
@@ -816,7 +846,8 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   }
 
   CUtensorMap ta, tb;
-  if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) || !tmap_kmajor(&tb, wb, h, v, h, kBBoxRows))
+  if (!tmap_kmajor(&ta, hidden, h, n, h, kBM) ||
+      !(fused ? tmap_kmajor_f32(&tb, weight, h, v, h) : tmap_kmajor(&tb, wb, h, v, h, kBBoxRows)))
     return FLCE_ERR_CUDA;
   const GemmProblem prob = make_problem(n, v, h, false, false, kEpiForward, dev->num_sms / 2);
   EpiSet<kEpiSetForward> es{};
@@ -835,10 +866,13 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   // run slower take fewer tiles and the launch does not wait on the slowest one.
   unsigned* counter = reinterpret_cast<unsigned*>(ws + p.off_cnt);
   if (cudaMemsetAsync(counter, 0, sizeof(unsigned), cs) != cudaSuccess) return FLCE_ERR_CUDA;
-  if ((st = launch_group<kEpiSetForward, ProblemCfg<false, false, kEpiForward>>(
-           &prob, &ta, &tb, 1, es, counter, *dev, cs, KF_GEMM_FWD, fwd_flops, fwd_bytes)) !=
-      FLCE_OK)
-    return st;
+  st = fused ? launch_group<kEpiSetForward, ProblemCfg<false, false, kEpiForward, true>>(
+                   &prob, &ta, &tb, 1, es, counter, *dev, cs, KF_GEMM_FWD, fwd_flops,
+                   fwd_bytes + 2.0 * double(v) * double(h))
+             : launch_group<kEpiSetForward, ProblemCfg<false, false, kEpiForward>>(
+                   &prob, &ta, &tb, 1, es, counter, *dev, cs, KF_GEMM_FWD, fwd_flops,
+                   fwd_bytes);
+  if (st != FLCE_OK) return st;
   {
     LaunchScope scope(KF_MERGE, 0.0, 8.0 * double(p.v_tiles) * n + 24.0 * n, cs);
     lse_merge_kernel<<<int(p.nblk), kMergeRows * kMergeWarps, 0, cs>>>(
@@ -855,6 +889,16 @@ extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
   return FLCE_OK;
 }
 
+extern "C" int flce_forward(const void* hidden, const void* weight, int w_dtype,
+                            const int64_t* labels, int64_t n, int64_t h, int64_t vp,
+                            int64_t unpadded, int64_t ignore_index, float softcap, int reduction,
+                            int64_t num_label_tokens, float* loss, float* lse, void* workspace,
+                            size_t ws_bytes, flce_stream_t stream) {
+  return flce_forward_ex(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index,
+                         softcap, reduction, num_label_tokens, loss, lse, workspace, ws_bytes, 0u,
+                         stream);
+}
+
 extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dtype,
                                 const int64_t* labels, int64_t n, int64_t h, int64_t vp,
                                 int64_t unpadded, int64_t ignore_index, float softcap,
@@ -866,14 +910,18 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   int st = check_common(hidden, weight, w_dtype, labels, n, h, vp, v, softcap, reduction,
                         num_label_tokens);
   if (st != FLCE_OK) return st;
-  if ((flags & ~FLCE_BWD_HEAD_COPY_VALID) != 0u) return FLCE_ERR_INVALID_ARG;
+  if ((flags & ~(FLCE_BWD_HEAD_COPY_VALID | FLCE_FUSED_HEAD_CAST)) != 0u ||
+      (flags & (FLCE_BWD_HEAD_COPY_VALID | FLCE_FUSED_HEAD_CAST)) ==
+          (FLCE_BWD_HEAD_COPY_VALID | FLCE_FUSED_HEAD_CAST))
+    return FLCE_ERR_INVALID_ARG;
+  const bool fused = (flags & FLCE_FUSED_HEAD_CAST) != 0u && w_dtype == FLCE_F32;
   if (dweight == nullptr || !aligned(dweight, 16)) return FLCE_ERR_INVALID_ARG;
   if (n > 0) {
     if (grad_loss == nullptr || lse == nullptr || dhidden == nullptr) return FLCE_ERR_INVALID_ARG;
     if (!aligned(grad_loss, 4) || !aligned(lse, 4) || !aligned(dhidden, 16))
       return FLCE_ERR_INVALID_ARG;
   }
-  const Shape s{n, h, vp, v, w_dtype};
+  const Shape s{n, h, vp, v, w_dtype, fused ? 1 : 0};
   const BwdPlan p0 = plan_backward(s, kBN);
   if (workspace == nullptr || !aligned(workspace, 16) || ws_bytes < p0.total)
     return FLCE_ERR_WORKSPACE;
@@ -900,7 +948,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   if (n == 0) return FLCE_OK;
 
   const void* wb = weight;
-  if (w_dtype == FLCE_F32) {
+  if (w_dtype == FLCE_F32 && !fused) {
     wb = ws + p.off_wb;
     // The caller vouches that the copy at offset 0 still holds bf16(weight[:V])
     // (written by flce_forward on this workspace and unchanged since).
@@ -926,13 +974,35 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
   CUtensorMap t_hid_k, t_w_k, t_hid_mn, t_w_mn;
-  if (!tmap_kmajor(&t_hid_k, hidden, h, n, h, kBM) || !tmap_kmajor(&t_w_k, wb, h, v, h, kBBoxRows) ||
-      !tmap_mnmajor(&t_hid_mn, hidden, h, n, h) || !tmap_mnmajor(&t_w_mn, wb, h, v, h))
+  if (!tmap_kmajor(&t_hid_k, hidden, h, n, h, kBM) || !tmap_mnmajor(&t_hid_mn, hidden, h, n, h))
+    return FLCE_ERR_CUDA;
+  if (fused ? !tmap_kmajor_f32(&t_w_k, weight, h, v, h) || !tmap_mnmajor_f32(&t_w_mn, weight, h, v, h)
+            : !tmap_kmajor(&t_w_k, wb, h, v, h, kBBoxRows) || !tmap_mnmajor(&t_w_mn, wb, h, v, h))
     return FLCE_ERR_CUDA;
 
-  using CfgGrad = ProblemCfg<false, false, kEpiGrad>;
-  using CfgDh = ProblemCfg<false, true, kEpiAccumRows>;
+  // The head's GEMMs (recompute: B = W K-major; dhidden: B = W MN-major) take
+  // it as FP32 and round it in the kernel when `fused`.
   using CfgDw = ProblemCfg<true, true, kEpiStoreRows>;
+  auto launch_grad = [&](const GemmProblem* pr, const CUtensorMap* ma, const CUtensorMap* mb,
+                         const EpiSet<kEpiSetBackward>& es, unsigned* cnt, double fl,
+                         double by) {
+    return fused ? launch_group<kEpiSetBackward, ProblemCfg<false, false, kEpiGrad, true>>(
+                       pr, ma, mb, 1, es, cnt, *dev, cs, KF_GEMM_GRAD, fl, by)
+                 : launch_group<kEpiSetBackward, ProblemCfg<false, false, kEpiGrad>>(
+                       pr, ma, mb, 1, es, cnt, *dev, cs, KF_GEMM_GRAD, fl, by);
+  };
+  auto launch_fused_bwd = [&](const GemmProblem* pr, const CUtensorMap* ma,
+                              const CUtensorMap* mb, int count,
+                              const EpiSet<kEpiSetBackward>& es, unsigned* cnt, double fl,
+                              double by) {
+    return fused ? launch_group<kEpiSetBackward, ProblemCfg<false, true, kEpiAccumRows, true>,
+                                CfgDw, ProblemCfg<false, false, kEpiGrad, true>>(
+                       pr, ma, mb, count, es, cnt, *dev, cs, KF_GEMM_BWD, fl, by)
+                 : launch_group<kEpiSetBackward, ProblemCfg<false, true, kEpiAccumRows>, CfgDw,
+                                ProblemCfg<false, false, kEpiGrad>>(
+                       pr, ma, mb, count, es, cnt, *dev, cs, KF_GEMM_BWD, fl, by);
+  };
+  const double w_extra = fused ? 2.0 : 0.0;  // FP32 head bytes beyond the BF16 ones
   const int64_t chunks = cdiv(v, vc);
   auto chunk_v0 = [&](int64_t c) { return c * vc; };
   auto chunk_width = [&](int64_t c) { return std::min(vc, v - c * vc); };
@@ -960,7 +1030,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   auto grad_flops = [&](int64_t c) { return 2.0 * double(n) * double(chunk_width(c)) * double(h); };
   auto grad_bytes = [&](int64_t c) {
     return 2.0 * (double(n) + double(chunk_width(c))) * double(h) +
-           2.0 * double(n) * double(chunk_gcols(c));
+           w_extra * double(chunk_width(c)) * double(h) + 2.0 * double(n) * double(chunk_gcols(c));
   };
 
   {  // K3 of the first chunk on its own
@@ -968,9 +1038,8 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     CUtensorMap ma, mb;
     EpiSet<kEpiSetBackward> es{};
     grad_problem(0, &pr, &ma, &mb, &es.grad);
-    if ((st = launch_group<kEpiSetBackward, CfgGrad>(&pr, &ma, &mb, 1, es, &counters[0], *dev, cs,
-                                                     KF_GEMM_GRAD, grad_flops(0),
-                                                     grad_bytes(0))) != FLCE_OK)
+    if ((st = launch_grad(&pr, &ma, &mb, es, &counters[0], grad_flops(0), grad_bytes(0))) !=
+        FLCE_OK)
       return st;
   }
   for (int64_t c = 0; c < chunks; ++c) {
@@ -998,7 +1067,8 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     {
       const double rmw = es.accum.mode == 0 ? 4.0 : (es.accum.mode == 1 ? 8.0 : (es.accum.mode == 2 ? 6.0 : 2.0));
       flops += 2.0 * double(n) * double(width) * double(h);
-      bytes += 2.0 * double(n) * gcols + 2.0 * double(width) * h + rmw * double(n) * h;
+      bytes += 2.0 * double(n) * gcols + (2.0 + w_extra) * double(width) * h +
+               rmw * double(n) * h;
     }
     ++count;
     // K4: dW[v0 : v0 + width] = G^T . hidden  (contraction over tokens)
@@ -1020,8 +1090,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
       bytes += grad_bytes(c + 1);
       ++count;
     }
-    if ((st = launch_group<kEpiSetBackward, CfgDh, CfgDw, CfgGrad>(
-             pr, ma, mb, count, es, &counters[c + 1], *dev, cs, KF_GEMM_BWD, flops, bytes)) !=
+    if ((st = launch_fused_bwd(pr, ma, mb, count, es, &counters[c + 1], flops, bytes)) !=
         FLCE_OK)
       return st;
   }
@@ -1191,8 +1260,11 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
   NvtxRange range("flce_forward_noalloc");
   const int64_t v = unpadded <= 0 ? vp : unpadded;
   if (!shape_ok(n, h, vp, v, w_dtype)) return FLCE_ERR_INVALID_ARG;
-  // The whole scratch must fit the fixed array; nothing here can grow it.
-  if (plan_forward(Shape{n, h, vp, v, w_dtype}).total > kNoAllocScratchBytes)
+  // An FP32 head is rounded inside the GEMM (no BF16 copy), so the scratch is
+  // the same as for a BF16 head; it must fit the fixed array, which nothing
+  // here can grow.
+  const unsigned flags = w_dtype == FLCE_F32 ? FLCE_FUSED_HEAD_CAST : 0u;
+  if (plan_forward(Shape{n, h, vp, v, w_dtype, flags != 0u ? 1 : 0}).total > kNoAllocScratchBytes)
     return FLCE_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FLCE_ERR_CUDA;
@@ -1216,9 +1288,9 @@ extern "C" int flce_forward_noalloc(const void* hidden, const void* weight, int 
   // Same kernels, same results as flce_forward; every scratch byte the
   // forward reads is written earlier in the same call, so the array's stale
   // contents from a previous call never need clearing.
-  return flce_forward(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index, softcap,
-                      reduction, num_label_tokens, loss, lse, scratch, kNoAllocScratchBytes,
-                      stream);
+  return flce_forward_ex(hidden, weight, w_dtype, labels, n, h, vp, unpadded, ignore_index,
+                         softcap, reduction, num_label_tokens, loss, lse, scratch,
+                         kNoAllocScratchBytes, flags, stream);
 }
 
 // ===================================== cross entropy on given logits (chunked_ce)

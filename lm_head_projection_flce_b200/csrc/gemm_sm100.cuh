@@ -20,6 +20,7 @@ constexpr int kBK = 64;       // K per stage: one 128-byte swizzle row of BF16
 constexpr int kUmmaK = 16;    // K per tcgen05.mma (kind::f16)
 constexpr int kThreads = 192; // warp 0 scheduler/loads, warp 1 MMA, warps 2..5 epilogue
 constexpr int kEpiWarps = 4;
+constexpr int kConvWarps = 8; // warps 6..13 of kernels with an FP32 B operand: the converter
 constexpr int kTmemCols = 512;
 constexpr int kSchedSlots = 4;
 constexpr int kMaxProblems = 3;
@@ -93,11 +94,17 @@ struct PipeCtl {
 };
 
 // Bounded wait: true once the phase completed; false on abort or timeout.
+// kCluster: acquire at cluster scope (the arrivals publish the peer CTA's
+// shared-memory stores).
+template <bool kCluster = false>
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, PipeCtl* ctl,
                                            unsigned* err, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() {
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (test()) return true;
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!test()) {
     if (ctl->abort) return false;
     if (global_timer_ns() - t0 > timeout_ns) {
       ctl->abort = 1;
@@ -117,17 +124,21 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 }
 
 // Compile-time configuration of one problem slot of a grouped launch.
-template <bool kAMnMajor, bool kBMnMajor, int kEpiKind>
+// kBF32: B is FP32 in global memory and is rounded to BF16 (nearest even) on
+// its way into shared memory by the kernel's converter warps.
+template <bool kAMnMajor, bool kBMnMajor, int kEpiKind, bool kBFp32 = false>
 struct ProblemCfg {
   static constexpr bool kAMn = kAMnMajor;
   static constexpr bool kBMn = kBMnMajor;
   static constexpr int kEpi = kEpiKind;
+  static constexpr bool kBF32 = kBFp32;
   static constexpr bool kValid = true;
 };
 struct NoProblem {
   static constexpr bool kAMn = false;
   static constexpr bool kBMn = false;
   static constexpr int kEpi = -1;
+  static constexpr bool kBF32 = false;
   static constexpr bool kValid = false;
 };
 

@@ -34,6 +34,7 @@ STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_INVALID_ARG", 2: "FLCE_ERR_WORKSPACE",
           6: "FLCE_ERR_TIMEOUT"}
 REDUCTIONS = {"sum": 0, "mean": 1, "none": 2}
 FLCE_BWD_HEAD_COPY_VALID = 1
+FLCE_FUSED_HEAD_CAST = 2
 W_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 _c_i64 = ctypes.c_int64
@@ -45,9 +46,15 @@ _c_size = ctypes.c_size_t
 SIGNATURES = {
     "flce_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int]),
     "flce_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int]),
+    "flce_workspace_size_ex": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int, ctypes.c_uint]),
+    "flce_workspace_min_size_ex": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_int,
+                                             ctypes.c_uint]),
     "flce_forward": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
                               _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr,
                               _c_size, _c_ptr]),
+    "flce_forward_ex": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64,
+                                 _c_i64, _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr,
+                                 _c_ptr, _c_size, ctypes.c_uint, _c_ptr]),
     "flce_backward": (_c_int, [_c_ptr, _c_ptr, _c_int, _c_ptr, _c_i64, _c_i64, _c_i64, _c_i64,
                                _c_i64, ctypes.c_float, _c_int, _c_i64, _c_ptr, _c_ptr, _c_ptr,
                                _c_ptr, _c_ptr, _c_size, _c_ptr]),
@@ -124,10 +131,12 @@ def _vocab(weight: torch.Tensor, unpadded_vocab: int | None) -> int:
 
 
 def workspace_size(n_tokens: int, hidden: int, padded_vocab: int, unpadded_vocab: int | None,
-                   w_dtype: torch.dtype = torch.bfloat16, minimum: bool = False) -> int:
+                   w_dtype: torch.dtype = torch.bfloat16, minimum: bool = False,
+                   fused_head_cast: bool = False) -> int:
     lib = load_library()
-    fn = lib.flce_workspace_min_size if minimum else lib.flce_workspace_size
-    return int(fn(n_tokens, hidden, padded_vocab, unpadded_vocab or 0, W_DTYPES[w_dtype]))
+    fn = lib.flce_workspace_min_size_ex if minimum else lib.flce_workspace_size_ex
+    return int(fn(n_tokens, hidden, padded_vocab, unpadded_vocab or 0, W_DTYPES[w_dtype],
+                  FLCE_FUSED_HEAD_CAST if fused_head_cast else 0))
 
 
 def _prepare(hidden, weight, labels):
@@ -182,8 +191,14 @@ def _forward_outputs(loss, lse, n: int, reduction: str, dev):
 def forward(hidden, weight, labels, *, ignore_index: int = -100, softcap: float = 0.0,
             unpadded_vocab: int | None = None, reduction: str = "sum",
             num_label_tokens: int | None = None, workspace: torch.Tensor | None = None,
-            loss: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
-    """Fused projection + cross entropy.  Returns ``(loss, lse)`` (FP32)."""
+            loss: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+            fused_head_cast: bool = False, stream=None):
+    """Fused projection + cross entropy.  Returns ``(loss, lse)`` (FP32).
+
+    ``fused_head_cast=True`` (flce_forward_ex with FLCE_FUSED_HEAD_CAST): an
+    FP32 head is rounded to BF16 inside the GEMM instead of into a V x H BF16
+    copy in the workspace; same results, smaller workspace, slower GEMM.
+    """
     lib = load_library()
     hid, lab = _prepare(hidden, weight, labels)
     n, h = hid.shape
@@ -192,10 +207,13 @@ def forward(hidden, weight, labels, *, ignore_index: int = -100, softcap: float 
     dev = hid.device
     red = REDUCTIONS[reduction]
     loss, lse = _forward_outputs(loss, lse, n, reduction, dev)
-    ws, ws_bytes = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
-    st = lib.flce_forward(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
-                          v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
-                          _ptr(loss), _ptr(lse), _ptr(ws), ws_bytes, _stream_handle(dev, stream))
+    ws, ws_bytes = _workspace(
+        workspace, workspace_size(n, h, vp, v, weight.dtype, fused_head_cast=fused_head_cast), dev)
+    st = lib.flce_forward_ex(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h, vp,
+                             v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
+                             _ptr(loss), _ptr(lse), _ptr(ws), ws_bytes,
+                             FLCE_FUSED_HEAD_CAST if fused_head_cast else 0,
+                             _stream_handle(dev, stream))
     _check("flce_forward", st)
     return (loss if reduction == "none" else loss.reshape(())), lse
 
@@ -213,7 +231,7 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
              softcap: float = 0.0, unpadded_vocab: int | None = None, reduction: str = "sum",
              num_label_tokens: int | None = None, workspace: torch.Tensor | None = None,
              dhidden: torch.Tensor | None = None, dweight: torch.Tensor | None = None,
-             reuse_head_copy: bool = False, stream=None):
+             reuse_head_copy: bool = False, fused_head_cast: bool = False, stream=None):
     """Gradients ``(dhidden [.., H] bf16, dweight [Vp, H] in the head's dtype)``.
 
     ``reuse_head_copy=True`` (flce_backward_ex with FLCE_BWD_HEAD_COPY_VALID):
@@ -221,6 +239,10 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
     ``forward`` wrote into the same ``workspace`` -- the caller promises that
     the head and that workspace are unchanged since.  Needs ``workspace``;
     ignored for a BF16 head.
+
+    ``fused_head_cast=True`` (FLCE_FUSED_HEAD_CAST): the recompute and
+    dhidden GEMMs round an FP32 head to BF16 inside the kernel; no copy is
+    read or written.  Not combinable with ``reuse_head_copy``.
     """
     lib = load_library()
     hid, lab = _prepare(hidden, weight, labels)
@@ -237,8 +259,12 @@ def backward(hidden, weight, labels, lse, grad_loss, *, ignore_index: int = -100
                else _buffer(dweight, weight.numel(), weight.dtype, dev, "dweight"))
     if reuse_head_copy and workspace is None:
         raise ValueError("reuse_head_copy needs the workspace the forward wrote the copy into")
-    ws, ws_bytes = _workspace(workspace, workspace_size(n, h, vp, v, weight.dtype), dev)
-    flags = FLCE_BWD_HEAD_COPY_VALID if reuse_head_copy else 0
+    if reuse_head_copy and fused_head_cast:
+        raise ValueError("fused_head_cast writes no head copy to reuse")
+    ws, ws_bytes = _workspace(
+        workspace, workspace_size(n, h, vp, v, weight.dtype, fused_head_cast=fused_head_cast), dev)
+    flags = (FLCE_BWD_HEAD_COPY_VALID if reuse_head_copy else 0) | (
+        FLCE_FUSED_HEAD_CAST if fused_head_cast else 0)
     st = lib.flce_backward_ex(_ptr(hid), _ptr(weight), W_DTYPES[weight.dtype], _ptr(lab), n, h,
                               vp, v, ignore_index, float(softcap), red, int(num_label_tokens or 0),
                               _ptr(grad), _ptr(lse), _ptr(dhidden), _ptr(dweight), _ptr(ws),
@@ -275,48 +301,54 @@ def selftest_wait_timeout(timeout_us: int, device=None) -> None:
 class _FusedLinearCE(torch.autograd.Function):
     @staticmethod
     def forward(ctx, hidden, weight, labels, ignore_index, softcap, unpadded_vocab, reduction,
-                num_label_tokens):
+                num_label_tokens, fused_head_cast):
         # An FP32 head's BF16 copy, made by the forward, is kept (in the
         # workspace) for the backward instead of being cast again; autograd's
         # version check refuses a backward after the head changed in place.
+        # With fused_head_cast there is no copy and nothing is kept.
         ws = None
-        if weight.dtype == torch.float32:
+        if weight.dtype == torch.float32 and not fused_head_cast:
             hid = hidden.reshape(-1, hidden.shape[-1])
             need = workspace_size(hid.shape[0], hid.shape[1], weight.shape[0],
                                   _vocab(weight, unpadded_vocab), weight.dtype)
             ws = torch.empty(max(need, 16), dtype=torch.uint8, device=hidden.device)
         loss, lse = forward(hidden, weight, labels, ignore_index=ignore_index, softcap=softcap,
                             unpadded_vocab=unpadded_vocab, reduction=reduction,
-                            num_label_tokens=num_label_tokens, workspace=ws)
+                            num_label_tokens=num_label_tokens, workspace=ws,
+                            fused_head_cast=fused_head_cast)
         ctx.save_for_backward(hidden, weight, labels, lse)
         ctx.workspace = ws
-        ctx.opts = (ignore_index, softcap, unpadded_vocab, reduction, num_label_tokens)
+        ctx.opts = (ignore_index, softcap, unpadded_vocab, reduction, num_label_tokens,
+                    fused_head_cast)
         return loss
 
     @staticmethod
     def backward(ctx, grad_out):
         hidden, weight, labels, lse = ctx.saved_tensors
-        ii, c, uv, red, nlt = ctx.opts
+        ii, c, uv, red, nlt, fused = ctx.opts
         ws = ctx.workspace
         ctx.workspace = None
         dh, dw = backward(hidden, weight, labels, lse, grad_out, ignore_index=ii, softcap=c,
                           unpadded_vocab=uv, reduction=red, num_label_tokens=nlt, workspace=ws,
-                          reuse_head_copy=ws is not None)
-        return dh, dw, None, None, None, None, None, None
+                          reuse_head_copy=ws is not None, fused_head_cast=fused)
+        return dh, dw, None, None, None, None, None, None, None
 
 
 def fused_linear_cross_entropy(hidden, weight, labels, *, ignore_index: int = -100,
                                softcap: float = 0.0, unpadded_vocab: int | None = None,
-                               reduction: str = "sum", num_label_tokens: int | None = None):
+                               reduction: str = "sum", num_label_tokens: int | None = None,
+                               fused_head_cast: bool = False):
     """Autograd-aware loss: gradients flow to ``hidden`` and ``weight``.
 
     With an FP32 head the forward's workspace (which holds the head's BF16
     copy, V x H x 2 bytes, and the backward's buffers) is kept until the
     backward runs, so the head is cast once per step; a BF16 head keeps
-    nothing between the two.
+    nothing between the two.  ``fused_head_cast=True`` rounds an FP32 head
+    inside the GEMMs instead: no copy exists and nothing is kept (less memory,
+    slower GEMMs, the same results).
     """
     return _FusedLinearCE.apply(hidden, weight, labels, ignore_index, softcap, unpadded_vocab,
-                                reduction, num_label_tokens)
+                                reduction, num_label_tokens, fused_head_cast)
 
 
 class CapturedStep:

@@ -141,13 +141,52 @@ def test_backward_ex_flags(lib):
                                     a["h"], a["vp"], a["v"], a["ii"], a["c"], a["red"], a["nlt"],
                                     a["grad"], a["lse"], a["dh"], a["dw"], a["ws"], a["ws_bytes"],
                                     flags, a["stream"])
-    assert bex(2) == 1 and bex(0x80000000) == 1 and bex(3) == 1   # unknown bits
+    assert bex(4) == 1 and bex(0x80000000) == 1                  # unknown bits
+    assert bex(3) == 1                          # reuse a copy and write none: contradictory
     assert bex(1, h=250) == 1 and bex(1, ws=0) == 2              # the usual checks stay
-    # the documented flag passes the host checks (then the missing GPU answers)
+    assert bex(2, h=250) == 1 and bex(2, ws=0) == 2
+    # the documented flags pass the host checks (then the missing GPU answers)
     import torch
     if not torch.cuda.is_available():
         assert bex(flce.FLCE_BWD_HEAD_COPY_VALID) in (3, 4)
+        assert bex(flce.FLCE_FUSED_HEAD_CAST) in (3, 4)
         assert bex(0) in (3, 4)
+
+
+def test_forward_ex_flags(lib):
+    def fex(flags, **kw):
+        a = dict(hidden=FAKE, weight=FAKE, w_dtype=1, labels=FAKE, n=64, h=256, vp=1024, v=1024,
+                 ii=-100, c=0.0, red=0, nlt=0, loss=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 40,
+                 stream=None)
+        a.update(kw)
+        return lib.flce_forward_ex(a["hidden"], a["weight"], a["w_dtype"], a["labels"], a["n"],
+                                   a["h"], a["vp"], a["v"], a["ii"], a["c"], a["red"], a["nlt"],
+                                   a["loss"], a["lse"], a["ws"], a["ws_bytes"], flags,
+                                   a["stream"])
+    assert fex(1) == 1 and fex(4) == 1 and fex(0x80000000) == 1  # only FLCE_FUSED_HEAD_CAST
+    assert fex(2, h=250) == 1 and fex(2, ws=0) == 2
+    import torch
+    if not torch.cuda.is_available():
+        assert fex(flce.FLCE_FUSED_HEAD_CAST) in (3, 4)
+        assert fex(0) in (3, 4)
+
+
+def test_workspace_size_without_the_head_copy(lib):
+    """FLCE_FUSED_HEAD_CAST drops exactly the FP32 head's BF16 copy (V x H x 2
+    bytes, rounded up to 1 KiB) from both sizes; a BF16 head has no copy."""
+    f32, bf16 = 1, 0
+    for n, h, vp, v in ((4096, 4096, 128256, 128256), (8192, 5376, 262144, 256000),
+                        (333, 328, 1024, 1000), (0, 8, 100, 0)):
+        vv = v if v > 0 else vp
+        copy = -(-vv * h * 2 // 1024) * 1024
+        for full in (lib.flce_workspace_size_ex, lib.flce_workspace_min_size_ex):
+            assert full(n, h, vp, v, f32, 0) - full(n, h, vp, v, f32, 2) == copy
+            assert full(n, h, vp, v, bf16, 0) == full(n, h, vp, v, bf16, 2)
+            assert full(n, h, vp, v, f32, 1) == 0 and full(n, h, vp, v, f32, 4) == 0
+        assert lib.flce_workspace_size_ex(n, h, vp, v, f32, 0) == \
+            lib.flce_workspace_size(n, h, vp, v, f32)
+        assert lib.flce_workspace_min_size_ex(n, h, vp, v, f32, 0) == \
+            lib.flce_workspace_min_size(n, h, vp, v, f32)
 
 
 def test_backward_specific_arguments(lib):
