@@ -55,6 +55,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the short timed passes of the other large workloads and of cross "
                          "entropy on given logits (one GPU only) under 'extra_workloads'")
+    ap.add_argument("--fused-head-cast", action="store_true",
+                    help="with an FP32 head, round it to BF16 inside the GEMMs "
+                         "(FLCE_FUSED_HEAD_CAST) instead of casting it into a copy")
     ap.add_argument("--extra-steps", type=int, default=5,
                     help="timed steps of each extra workload (at least 5)")
     ap.add_argument("--path", choices=["flce", "chunked_ce"], default="flce",
@@ -610,6 +613,10 @@ def run_ours(args, w) -> int:
     warmup = max(args.warmup, 3)
 
     run = FlceRun(w, dev, graph=args.graph)
+    if args.fused_head_cast:
+        if args.graph or w.w_dtype != "f32":
+            raise SystemExit("--fused-head-cast needs an FP32-head workload and no --graph")
+        run.use_fused_head_cast(dev)
     n = w.n_tokens
 
     # ---- end to end: pinned host inputs -> device, fwd + bwd, loss -> host, every step.
@@ -681,7 +688,8 @@ def run_ours(args, w) -> int:
             "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**workload_config(w, f"replicas x{world} (one independent batch per GPU)"),
-                       **({"cuda_graph": True} if args.graph else {})},
+                       **({"cuda_graph": True} if args.graph else {}),
+                       **({"head_cast": "fused into the GEMMs"} if run.fused_cast else {})},
             "roofline": m["roofline"],
             "kernels": m["kernels"],
             "kernel_timing": ("per-launch CUDA events in a second pass of the same steps"
