@@ -31,6 +31,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 32 FP32 values rounded to BF16 and stored at `out` (64 bytes): two 32-byte
+// stores when `v8` (out 32-byte aligned), else four 16-byte ones.
+__device__ __forceinline__ void store_bf16x32(uint4* out, const float (&v)[32], bool v8) {
+  if (v8) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      st_global_v8(out + 2 * q, pack_bf16x2(v[16 * q + 0], v[16 * q + 1]),
+                   pack_bf16x2(v[16 * q + 2], v[16 * q + 3]),
+                   pack_bf16x2(v[16 * q + 4], v[16 * q + 5]),
+                   pack_bf16x2(v[16 * q + 6], v[16 * q + 7]),
+                   pack_bf16x2(v[16 * q + 8], v[16 * q + 9]),
+                   pack_bf16x2(v[16 * q + 10], v[16 * q + 11]),
+                   pack_bf16x2(v[16 * q + 12], v[16 * q + 13]),
+                   pack_bf16x2(v[16 * q + 14], v[16 * q + 15]));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      out[q] = w;
+    }
+  }
+}
+
 // -------------------------------------------------------------------------
 // Forward: logits tile -> per-row partial (max, sum of exponentials) over the
 // tile's live vocabulary columns, plus the label's capped logit.
@@ -145,6 +172,7 @@ struct EpiGrad {
     const float* scale;  // [n_tokens] d loss / d token loss (0 if ignored)
     __nv_bfloat16* g;    // [n_tokens][ldg]
     int64_t ldg;
+    int v8;              // 1: g and its rows are 32-byte aligned (32-byte stores)
   };
 
   static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
@@ -213,17 +241,7 @@ struct EpiGrad {
         for (int j = 0; j < 32; ++j)
           if (c0 + j >= ncols) v[j] = 0.0f;
       }
-      if (live) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-          w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-          w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-          w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-          out[c0 / 8 + q] = w;
-        }
-      }
+      if (live) store_bf16x32(out + c0 / 8, v, p.v8 != 0);
     }
   }
 };
@@ -240,6 +258,7 @@ struct EpiStoreRows {
     int64_t rows;
     int64_t cols;
     int f32;
+    int v8;      // 1: out and its rows are 32-byte aligned (32-byte stores)
   };
 
   static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
@@ -252,6 +271,22 @@ struct EpiStoreRows {
       float v[32];
       tmem_load_32cols(taddr + c0, v);
       if (!live) continue;
+      if (p.v8 && h0 + c0 + 32 <= p.cols) {  // all 32 columns in range
+        if (p.f32) {
+          float* o = static_cast<float*>(p.out) + r * p.ldo + h0 + c0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_global_v8(o + 8 * q, __float_as_uint(v[8 * q + 0]), __float_as_uint(v[8 * q + 1]),
+                         __float_as_uint(v[8 * q + 2]), __float_as_uint(v[8 * q + 3]),
+                         __float_as_uint(v[8 * q + 4]), __float_as_uint(v[8 * q + 5]),
+                         __float_as_uint(v[8 * q + 6]), __float_as_uint(v[8 * q + 7]));
+        } else {
+          store_bf16x32(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + r * p.ldo +
+                                                 h0 + c0),
+                        v, true);
+        }
+        continue;
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int64_t h = h0 + c0 + 8 * q;
@@ -288,6 +323,7 @@ struct EpiAccumRows {
     int64_t rows;
     int64_t cols;          // multiple of 8
     int mode;
+    int v8;                // 1: acc32 and its rows are 32-byte aligned (32-byte accesses)
   };
 
   static __device__ __forceinline__ void tile(const Params& p, uint32_t taddr, int mt, int nt,
@@ -309,14 +345,27 @@ struct EpiAccumRows {
 #pragma unroll
         for (int i = 0; i < 8; ++i) x[i] = v[8 * q + i];
         if (p.mode == 1 || p.mode == 2) {
-          const float4 a0 = reinterpret_cast<const float4*>(a)[0];
-          const float4 a1 = reinterpret_cast<const float4*>(a)[1];
-          x[0] += a0.x; x[1] += a0.y; x[2] += a0.z; x[3] += a0.w;
-          x[4] += a1.x; x[5] += a1.y; x[6] += a1.z; x[7] += a1.w;
+          if (p.v8) {
+            float y[8];
+            ld_global_v8(a, y);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] += y[i];
+          } else {
+            const float4 a0 = reinterpret_cast<const float4*>(a)[0];
+            const float4 a1 = reinterpret_cast<const float4*>(a)[1];
+            x[0] += a0.x; x[1] += a0.y; x[2] += a0.z; x[3] += a0.w;
+            x[4] += a1.x; x[5] += a1.y; x[6] += a1.z; x[7] += a1.w;
+          }
         }
         if (p.mode <= 1) {
-          reinterpret_cast<float4*>(a)[0] = make_float4(x[0], x[1], x[2], x[3]);
-          reinterpret_cast<float4*>(a)[1] = make_float4(x[4], x[5], x[6], x[7]);
+          if (p.v8) {
+            st_global_v8(a, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
+                         __float_as_uint(x[3]), __float_as_uint(x[4]), __float_as_uint(x[5]),
+                         __float_as_uint(x[6]), __float_as_uint(x[7]));
+          } else {
+            reinterpret_cast<float4*>(a)[0] = make_float4(x[0], x[1], x[2], x[3]);
+            reinterpret_cast<float4*>(a)[1] = make_float4(x[4], x[5], x[6], x[7]);
+          }
         } else {
           uint4 w;
           w.x = pack_bf16x2(x[0], x[1]);

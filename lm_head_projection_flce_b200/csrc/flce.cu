@@ -964,6 +964,9 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
   unsigned* counters = reinterpret_cast<unsigned*>(ws + p.off_cnt);
   __nv_bfloat16* gbufs[2] = {reinterpret_cast<__nv_bfloat16*>(ws + p.off_g),
                              reinterpret_cast<__nv_bfloat16*>(ws + p.off_g) + size_t(n) * vc};
+  // The chunk buffers' rows are vc x 2 bytes apart (vc % 256 == 0), so both
+  // buffers take 32-byte stores when the first starts 32-byte aligned.
+  const int g_v8 = aligned(gbufs[0], 32) ? 1 : 0;
   {
     LaunchScope prep_scope(KF_BWD_PREP, 0.0, 24.0 * double(n), cs);
     bwd_prep_kernel<<<1, 1024, 0, cs>>>(labels, nullptr, n, v, ignore_index, reduction,
@@ -1026,6 +1029,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     ep->scale = scale;
     ep->g = gbufs[c & 1];
     ep->ldg = vc;
+    ep->v8 = g_v8;
   };
   auto grad_flops = [&](int64_t c) { return 2.0 * double(n) * double(chunk_width(c)) * double(h); };
   auto grad_bytes = [&](int64_t c) {
@@ -1064,6 +1068,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     es.accum.rows = n;
     es.accum.cols = h;
     es.accum.mode = chunks == 1 ? 3 : (c == 0 ? 0 : (c == chunks - 1 ? 2 : 1));
+    es.accum.v8 = aligned(dh32, 32) ? 1 : 0;  // rows are H x 4 bytes apart, H % 8 == 0
     {
       const double rmw = es.accum.mode == 0 ? 4.0 : (es.accum.mode == 1 ? 8.0 : (es.accum.mode == 2 ? 6.0 : 2.0));
       flops += 2.0 * double(n) * double(width) * double(h);
@@ -1080,6 +1085,7 @@ extern "C" int flce_backward_ex(const void* hidden, const void* weight, int w_dt
     es.store.rows = width;
     es.store.cols = h;
     es.store.f32 = w_dtype == FLCE_F32;
+    es.store.v8 = aligned(es.store.out, 32) && (size_t(h) * wsz) % 32 == 0 ? 1 : 0;
     flops += 2.0 * double(n) * double(width) * double(h);
     bytes += 2.0 * double(n) * (double(gcols) + double(h)) + double(wsz) * width * h;
     ++count;
@@ -1149,6 +1155,7 @@ extern "C" int flce_selftest_gemm(const void* a, const void* b, float* d, int64_
   ep.rows = m;
   ep.cols = n;
   ep.f32 = 1;
+  ep.v8 = aligned(d, 32) ? 1 : 0;  // rows are n x 4 bytes apart, n % 8 == 0
   const double fl = 2.0 * double(m) * double(n) * double(k);
   const double by = 2.0 * (double(m) + double(n)) * double(k) + 4.0 * double(m) * n;
   const int f = KF_SELFTEST_GEMM;

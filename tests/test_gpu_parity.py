@@ -496,3 +496,35 @@ def test_matches_torch_cross_entropy_on_fp32_logits(dev, name):
     for got, want in ((dh.float(), h32.grad), (dw.float(), w32.grad)):
         scale = float(want.abs().max())
         assert float((got - want).abs().max()) <= GRAD_REL * scale
+
+
+@pytest.mark.parametrize("w_dtype", ["bf16", "f32"])
+def test_buffers_only_16_byte_aligned_take_the_16_byte_stores(dev, w_dtype):
+    """The G chunk, dW and dhidden-accumulator epilogues use 32-byte stores
+    when their buffer and its rows are 32-byte aligned, else 16-byte ones (the
+    ABI only asks for 16).  A workspace and outputs placed 16 bytes past a
+    32-byte boundary take the second path; every result equals the first's
+    bit for bit."""
+    # H = 528: rows are 32-byte multiples, and the last 32 columns of a 256-wide
+    # tile run past H (that chunk always takes the 16-byte stores)
+    w = W.custom(520, 528, 3000, 3072, w_dtype=w_dtype, softcap=30.0, ignore_frac=0.1, seed=41)
+    d = W.generate(w)
+    hid, wt, lab = (d[k].to(dev) for k in ("hidden", "weight", "labels"))
+    kw = dict(softcap=w.softcap, unpadded_vocab=w.vocab)
+    size = flce.workspace_size(w.n_tokens, w.hidden, w.padded_vocab, w.vocab, wt.dtype)
+    grad = torch.ones(1, device=dev)
+
+    def run(offset):
+        ws = torch.empty(size + 64, dtype=torch.uint8, device=dev)[offset:offset + size]
+        dwb = torch.empty(wt.numel() + 16, dtype=wt.dtype, device=dev)
+        dw = dwb[16 // wt.element_size() if offset else 0:][:wt.numel()].view(wt.shape)
+        assert (ws.data_ptr() % 32 == 0) == (offset == 0)
+        assert (dw.data_ptr() % 32 == 0) == (offset == 0)
+        loss, lse = flce.forward(hid, wt, lab, workspace=ws, **kw)
+        dh, dw = flce.backward(hid, wt, lab, lse, grad, workspace=ws, dweight=dw, **kw)
+        torch.cuda.synchronize(dev)
+        assert flce.get_error(dev) == flce.FLCE_OK
+        return loss.clone(), lse.clone(), dh.clone(), dw.clone()
+
+    for x, y in zip(run(0), run(16)):
+        assert torch.equal(x, y)
