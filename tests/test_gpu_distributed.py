@@ -18,7 +18,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(port, out, head_dtype="bf16"):
+def _worker(port, out, head_dtype="bf16", fused_head_cast=False):
     import sys
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -44,7 +44,7 @@ def _worker(port, out, head_dtype="bf16"):
         dt.requires_grad_(True)
         loss = data_parallel_fused_linear_cross_entropy(
             hid, dt, lab, num_label_tokens=d["num_label_tokens"], grad_reduce_group=dist.group.WORLD,
-            softcap=w.softcap, unpadded_vocab=w.vocab)
+            softcap=w.softcap, unpadded_vocab=w.vocab, fused_head_cast=fused_head_cast)
         loss.backward()
         h2 = d["hidden"].to(dev).requires_grad_(True)
         w2 = d["weight"].to(dev).requires_grad_(True)
@@ -59,16 +59,17 @@ def _worker(port, out, head_dtype="bf16"):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("head_dtype", ["bf16", "f32"])
-def test_data_parallel_wrapper_single_rank_nccl(head_dtype):
+@pytest.mark.parametrize("head_dtype,fused", [("bf16", False), ("f32", False), ("f32", True)])
+def test_data_parallel_wrapper_single_rank_nccl(head_dtype, fused):
     """The wrapper over a one-rank group equals the plain fused loss bit for bit,
     for a BF16 head and for FP32 master weights (whose BF16 copy the autograd
-    wrapper keeps from the forward for the backward)."""
+    wrapper keeps from the forward for the backward, or which the GEMMs round
+    in the kernel with fused_head_cast)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    p = ctx.Process(target=_worker, args=(_free_port(), q, head_dtype))
+    p = ctx.Process(target=_worker, args=(_free_port(), q, head_dtype, fused))
     p.start()
     p.join(timeout=300)
     assert p.exitcode == 0
