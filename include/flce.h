@@ -89,7 +89,9 @@ size_t flce_workspace_min_size(int64_t n_tokens, int64_t hidden, int64_t padded_
  * rounding as the copy) in shared memory, inside the kernel.  Results are
  * bit-identical to the copy's; the workspace shrinks by the copy, and the
  * GEMMs move twice the head bytes and convert every head tile once per tile
- * row, so they run slower than the copy path (measured in the design notes).
+ * row, so they run slower than the copy path: on one B200, 8192 tokens with
+ * H = 5376 and V = 256000 take about twice as long per forward + backward
+ * (0.51x the tokens/s) in a workspace of 1.85 GB instead of 4.61 GB.
  * The flag has no effect with a BF16 head.
  * The _ex sizes take the same flags (0 or FLCE_FUSED_HEAD_CAST; any other
  * bit gives 0).

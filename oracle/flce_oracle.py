@@ -24,7 +24,7 @@ What is computed, and where the pages fix it:
   head; the softmax is recomputed rather than stored
   ("nemo_automodel.components.loss.chunked_ce", _ChunkedCrossEntropySum.backward).
 
-Readings taken where the pages are silent (each also listed in the design notes):
+Readings taken where the pages are silent:
 softcap is ``c*tanh(z/c)`` with ``c = 0`` meaning off; logits are not rounded
 to BF16 before the softcap; a label outside ``[0, unpadded_vocab)`` that is not
 ``ignore_index`` is invalid (this oracle raises); labels are not shifted;
