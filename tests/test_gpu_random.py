@@ -71,6 +71,19 @@ def test_random_case(dev, i):
     rdh, rdw = O.backward(d["hidden"].double().numpy(), hw, labels.numpy(),
                           grad_loss=grad.double().numpy(), **kw)
     assert_parity(got, {"loss": np.asarray(fwd.loss), "lse": fwd.lse, "dh": rdh, "dw": rdw}), c
+    if wdt == torch.float32:
+        # The head rounded inside the GEMMs instead: a workspace smaller by exactly the
+        # copy keeps the same vocabulary chunking, so every result matches bit for bit.
+        copy = -(-c["v"] * c["h"] * 2 // 1024) * 1024
+        ws_f = torch.empty(max(ws_bytes - copy, 16), dtype=torch.uint8, device=dev)
+        kw_f = dict(ignore_index=c["ignore_index"], softcap=c["softcap"], unpadded_vocab=c["v"],
+                    reduction=red, num_label_tokens=nlt, workspace=ws_f, fused_head_cast=True)
+        loss_f, lse_f = flce.forward(hid, wt, lab, **kw_f)
+        dh_f, dw_f = flce.backward(hid, wt, lab, lse_f, grad.to(dev), **kw_f)
+        torch.cuda.synchronize(dev)
+        assert flce.get_error(dev) == flce.FLCE_OK
+        for x, y in ((loss, loss_f), (lse, lse_f), (dh, dh_f), (dw, dw_f)):
+            assert torch.equal(x, y), c
 
 
 def _draw_ce(i):
